@@ -1,0 +1,456 @@
+#!/usr/bin/env python3
+"""Benchmark of the absorbed-MLA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole path over the video-chunk workload (batch 1,
+n_h=32, d_h=128, d_c=512, d_R=64 3-D RoPE, 30x52-token frames, a 3-frame window plus a
+1-frame query chunk, hidden 4096, bf16): the chunk frame's cache write, query
+absorption, absorbed attention over the 6240-key window, and the W_UV up-projection.
+The ring holds the three window frames before timing starts.  Each rank runs its own
+independent sequence (weak scaling, no data-path collective).
+
+Printed metric: algorithmic TFLOP/s of the step (absorbed flops: per visible
+(query, key, head) 2(d_c+d_R) + 2 d_c, plus the three GEMMs), with
+the dominant kernel's roofline, the decode workload's latent-cache GB/s, an end-to-end
+figure through host buffers, and the CPU oracle baseline.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import configs as C  # noqa: E402
+from synth import generate as G  # noqa: E402
+
+WORKLOAD = C.VIDEO_CHUNK
+L2_FLUSH_BYTES = 256 << 20           # > 126 MB L2: written between timed steps
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ work accounting
+
+
+def visible_pairs(wl) -> int:
+    """(query, key) pairs the frame-block-causal mask keeps, summed over the batch."""
+    F = wl.tokens_per_frame
+    k_end = wl.k_first_tok + wl.n_keys
+    total = 0
+    for i in range(wl.n_queries):
+        g = wl.q_first_tok + i
+        total += min(k_end, (g // F + 1) * F) - wl.k_first_tok
+    return total * wl.batch
+
+
+def step_flops(wl) -> dict:
+    T, B = wl.n_queries, wl.batch
+    return {
+        "cache_write": 0 if wl.cache_direct else 2 * B * T * wl.d_model * wl.row_width,
+        "absorb_q": 2 * B * T * wl.n_heads * wl.d_nope * wl.d_latent,
+        "attend": visible_pairs(wl) * wl.n_heads * (2 * wl.row_width + 2 * wl.d_latent),
+        "up_v": 2 * B * T * wl.n_heads * wl.d_latent * wl.d_nope,
+    }
+
+
+def decode_bytes(wl) -> int:
+    """Algorithmic bytes of one decode attention call: every cached row read once,
+    q_abs read, o_lat and the LSE written."""
+    e = wl.elem_bytes
+    rows = wl.batch * wl.n_keys * wl.row_width * e
+    q = wl.batch * wl.n_heads * wl.row_width * e
+    o = wl.batch * wl.n_heads * wl.d_latent * e + wl.batch * wl.n_heads * 4
+    return rows + q + o
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+
+
+class Step:
+    """Device-resident state of one sequence's video-chunk step."""
+
+    def __init__(self, wl, seed, torch, mla):
+        self.wl, self.torch, self.mla = wl, torch, mla
+        dev = "cuda"
+        self.shape = mla.make_shape(wl)
+
+        def up(t):
+            return torch.from_numpy(t.storage.view(np.int16)).to(dev).view(torch.bfloat16)
+
+        w = G.weights(wl, seed)
+        self.w = {k: up(v) for k, v in w.items()}
+        F = wl.tokens_per_frame
+        self.cache = torch.zeros((wl.batch, wl.ring_slots, wl.row_width), dtype=torch.bfloat16,
+                                 device=dev)
+        first = wl.first_chunk_frame
+        for f in range(first):                       # the window, written before timing
+            h = up(G.hidden_frame(wl, seed, f))
+            mla.mla_cache_write(self.shape, h, wl.d_model, F, f * F, self.w["w_dkv"],
+                                self.w["w_kr"], self.cache)
+        hq = G.hidden_frames(wl, seed, first, wl.chunk_frames)
+        q = G.queries(wl, seed)
+        self.host = {"h": hq.storage.view(np.int16), "q_nope": q["q_nope"].storage.view(np.int16),
+                     "q_rope": q["q_rope"].storage.view(np.int16)}
+        self.dev_in = {k: torch.from_numpy(v).to(dev).view(torch.bfloat16)
+                       for k, v in self.host.items()}
+        self.pinned = {k: torch.from_numpy(v).pin_memory() for k, v in self.host.items()}
+        T = wl.n_queries
+        self.q_abs = torch.empty((wl.batch, T, wl.n_heads, wl.row_width), dtype=torch.bfloat16,
+                                 device=dev)
+        self.o_lat = torch.empty((wl.batch, T, wl.n_heads, wl.d_latent), dtype=torch.bfloat16,
+                                 device=dev)
+        self.lse = torch.empty((wl.batch, T, wl.n_heads), dtype=torch.float32, device=dev)
+        self.out = torch.empty((wl.batch, T, wl.n_heads, wl.d_nope), dtype=torch.bfloat16,
+                               device=dev)
+        self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
+        self.ws_bytes = mla.mla_attend_workspace_size(self.shape, T, wl.n_keys)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.ev_attend = []
+
+    def run(self, inp=None, attend_events=None):
+        wl, mla = self.wl, self.mla
+        inp = inp or self.dev_in
+        T = wl.n_queries
+        F = wl.tokens_per_frame
+        mla.mla_cache_write(self.shape, inp["h"], wl.d_model, T, wl.first_chunk_frame * F,
+                            self.w["w_dkv"], self.w["w_kr"], self.cache)
+        mla.mla_absorb_q(self.shape, inp["q_nope"], inp["q_rope"], T, wl.q_first_tok,
+                         self.w["w_uk"], self.q_abs)
+        if attend_events is not None:
+            attend_events[0].record()
+        mla.mla_attend(self.shape, self.q_abs, T, wl.q_first_tok, self.cache, wl.k_first_tok,
+                       wl.n_keys, wl.softmax_scale, self.o_lat, self.lse, self.ws, self.ws_bytes)
+        if attend_events is not None:
+            attend_events[1].record()
+        mla.mla_up_v(self.shape, self.o_lat, T, self.w["w_uv"], self.out)
+
+    def run_e2e(self):
+        """Host buffers in, host buffer out: copies inside the timed region."""
+        for k, v in self.pinned.items():
+            self.dev_in[k].view(torch_int16(self.torch)).copy_(v, non_blocking=True)
+        self.run()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+
+def torch_int16(torch):
+    return torch.int16
+
+
+def time_steps(torch, fn, steps, flush, with_attend=False):
+    """Per step: flush L2 (untimed), then CUDA events around the step on the current
+    stream.  Returns (step ms list, attend ms list)."""
+    st, at = [], []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) \
+            if with_attend else None
+        e0.record()
+        fn(a)
+        e1.record()
+        torch.cuda.synchronize()
+        st.append(e0.elapsed_time(e1))
+        if a:
+            at.append(a[0].elapsed_time(a[1]))
+    return st, at
+
+
+def decode_leg(torch, mla, steps, warmup, flush):
+    wl = C.DECODE
+    shape = mla.make_shape(wl)
+    dev = "cuda"
+    cache = torch.from_numpy(G.direct_cache(wl, 0).storage.view(np.int16)).to(dev).view(
+        torch.bfloat16)
+    q = G.queries(wl, 0)
+    w = G.weights(wl, 0)
+    up = lambda t: torch.from_numpy(t.storage.view(np.int16)).to(dev).view(torch.bfloat16)
+    q_abs = torch.empty((wl.batch, 1, wl.n_heads, wl.row_width), dtype=torch.bfloat16, device=dev)
+    mla.mla_absorb_q(shape, up(q["q_nope"]), up(q["q_rope"]), 1, wl.q_first_tok, up(w["w_uk"]),
+                     q_abs)
+    o_lat = torch.empty((wl.batch, 1, wl.n_heads, wl.d_latent), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, 1, wl.n_heads), dtype=torch.float32, device=dev)
+    nws = mla.mla_attend_workspace_size(shape, 1, wl.n_keys)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+
+    def call(_a=None):
+        mla.mla_attend(shape, q_abs, 1, wl.q_first_tok, cache, wl.k_first_tok, wl.n_keys,
+                       wl.softmax_scale, o_lat, lse, ws, nws)
+
+    for _ in range(warmup):
+        call()
+    ms, _ = time_steps(torch, call, steps, flush)
+    t = statistics.mean(ms)
+    return {"workload": wl.name, "value": decode_bytes(wl) / (t * 1e-3) / 1e9, "unit": "GB/s",
+            "ms": t, "bytes": decode_bytes(wl),
+            "tflops": step_flops(wl)["attend"] / (t * 1e-3) / 1e12}
+
+
+def cpu_baseline(seconds: float = 12.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the same step: the cache
+    write, absorption, absorbed attention and up-projection of a prefix of the chunk's
+    queries (all heads), repeated until ``seconds`` elapse."""
+    import oracle.mla_oracle as O
+    wl = WORKLOAD
+    w = {k: v.values for k, v in G.weights(wl, 0).items()}
+    F = wl.tokens_per_frame
+    rng_cache = np.zeros((wl.batch, wl.ring_slots, wl.row_width))
+    # window rows from the oracle's own cache write (not timed)
+    for f in range(wl.first_chunk_frame):
+        h = G.hidden_frame(wl, 0, f).values
+        rng_cache, _ = O.cache_write(rng_cache, h, w["w_dkv"], w["w_kr"], f * F, wl)
+    hq = G.hidden_frame(wl, 0, wl.first_chunk_frame).values
+    q = G.queries(wl, 0)
+    qn, qr = q["q_nope"].values, q["q_rope"].values
+    n_q = 0
+    flops = 0
+    t0 = time.perf_counter()
+    chunk = 8
+    while time.perf_counter() - t0 < seconds and n_q < wl.n_queries:
+        sl = slice(n_q, n_q + chunk)
+        n = min(chunk, wl.n_queries - n_q)
+        c2, _ = O.cache_write(rng_cache, hq[:, sl], w["w_dkv"], w["w_kr"], wl.q_first_tok + n_q, wl)
+        qa = O.absorb_q(qn[:, sl], qr[:, sl], w["w_uk"], wl.q_first_tok + n_q, wl)
+        lat, _ = O.attend_latent(qa, c2, wl.q_first_tok + n_q, wl.k_first_tok, wl.n_keys,
+                                 wl.softmax_scale, wl)
+        O.up_v(lat, w["w_uv"])
+        n_q += n
+        per_q = step_flops(wl)
+        flops += n * sum(per_q.values()) / wl.n_queries
+    dt = time.perf_counter() - t0
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        threads = max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n_q} of {wl.n_queries} chunk queries (all {wl.n_heads} heads, "
+                      f"{wl.n_keys} keys): cache write, absorption, latent attention, "
+                      f"up-projection in fp64 NumPy; {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import latent_kv_cache_write_b200 as mla
+    from latent_kv_cache_write_b200 import build
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus > 1 or world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    wl = WORKLOAD
+    step = Step(wl, seed=rank, torch=torch, mla=mla)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    assert mla.mla_device_error() == 0
+    n0 = mla.mla_kernel_launches()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ms, attend_ms = time_steps(torch, lambda a: step.run(attend_events=a), args.steps, flush,
+                                   with_attend=True)
+    torch.cuda.synchronize()
+    launches = mla.mla_kernel_launches() - n0
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(ms)
+    t_max = total_ms
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    # end to end through host buffers
+    for _ in range(max(1, args.warmup // 2)):
+        step.run_e2e()
+    e2e_ms, _ = time_steps(torch, lambda a: step.run_e2e(), args.steps, flush)
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    fl = step_flops(wl)
+    flops_step = sum(fl.values())
+    ms_step = t_max / args.steps
+    value = world * flops_step * args.steps / (t_max * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    att_ms = statistics.mean(attend_ms)
+    achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    dec = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush) if rank == 0 else None
+    if dec:
+        dec["peak_gbs"] = float(peaks["hbm_gbs"])
+        dec["frac"] = dec["value"] / dec["peak_gbs"]
+    if rank == 0:
+        line = {
+            "metric": "absorbed MLA attention TFLOP/s (chunk) and latent-cache GB/s (decode) "
+                      "vs B200 peak",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "n_heads": wl.n_heads,
+                       "d_nope": wl.d_nope, "d_latent": wl.d_latent, "d_rope": wl.d_rope,
+                       "frame": f"{wl.grid_h}x{wl.grid_w}", "window_frames": wl.window_frames,
+                       "chunk_frames": wl.chunk_frames, "keys": wl.n_keys,
+                       "queries": wl.n_queries, "d_model": wl.d_model,
+                       "step": "cache_write+absorb_q+attend+up_v",
+                       "flops_per_step": flops_step, "l2": "flushed (256 MB write) before each step",
+                       "parallelism": f"replicas x{world} (independent sequences)"},
+            "roofline": {"kernel": "mla_attend", "bound": "tensor", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "traffic": None, "ms_per_launch": att_ms},
+            "e2e": {"value": world * flops_step * args.steps / (e2e_total * 1e-3) / 1e12,
+                    "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(sum(v.nbytes for v in step.host.values())),
+                    "d2h_bytes_per_step": int(step.out.numel() * 2),
+                    "ms_per_step": e2e_total / args.steps},
+            "gpu_launches": int(launches),
+            "decode": dec,
+            "clocks": clocks.summary(),
+            "kernels_ms": {"attend": att_ms},
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores, on a bounded sample of
+    the same workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step_s = 4.0
+    for _ in range(args.warmup):
+        cpu_baseline(seconds=0.5)
+    vals, secs = [], 0.0
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(seconds=per_step_s)
+        vals.append(last["value"])
+        secs += last["seconds"]
+    v = statistics.mean(vals)
+    wl = WORKLOAD
+    line = {
+        "impl": "reference",
+        "metric": "absorbed MLA attention TFLOP/s (chunk) and latent-cache GB/s (decode) "
+                  "vs B200 peak",
+        "value": v, "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "kind": "oracle",
+                         "cores": last["cores"], "sample": last["sample"]},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+/*
+ * mla.h — C ABI of the absorbed multi-head latent attention hot path over a
+ * sliding-window latent KV ring, for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources cited by page title and section):
+ *   - Only a shared low-rank content latent c_KV (d_latent wide) and a shared
+ *     decoupled RoPE key k_R (d_rope wide) are cached per token
+ *     ("Multi-Head Latent Attention" concept page, "Low-rank joint compression" and
+ *     "The RoPE problem, and the decoupled fix"; "Understanding Multi-Head Latent
+ *     Attention and KV Compression", "Decoupling Rotary Position Embeddings (RoPE)").
+ *   - The positional key encodes the 3-D (t, h, w) position of a video token with
+ *     RoPE and the cache is a fixed-size sliding window over frames ("VideoMLA:
+ *     Compressing Video Diffusion Memory by 92.7% with Low-Rank Latent Attention",
+ *     "The Gap" and "Core Mechanism").
+ *   - W_UK is absorbed into the query, so scores are taken against the latent
+ *     directly; W_UV is applied after attention (concept page, "Low-rank joint
+ *     compression": the absorption identity).
+ *
+ * Conventions shared by every call
+ *   - Tensor arguments are DEVICE pointers to dense row-major arrays, 16-byte
+ *     aligned, in the storage dtype of the shape (float32 or bfloat16) unless stated.
+ *     The caller allocates and owns every buffer, workspace included; the library
+ *     allocates nothing and keeps no per-call state.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *     and the call returns without synchronising.  Results are visible to later work
+ *     on the same stream.
+ *   - Arguments are validated before anything is launched; on any error status no
+ *     work has been enqueued.  MLA_ERR_CUDA reports a launch failure
+ *     (cudaGetLastError after the launch).
+ *   - Positions: global token g lies in frame t = g / F (F = grid_h * grid_w), row
+ *     y = (g % F) / grid_w and column x = g % grid_w of that frame, and in ring slot
+ *     g mod ring_slots.  A one-token frame (grid 1x1) gives plain token positions
+ *     (1-D RoPE with rope_pairs = {d_rope/2, 0, 0}) and a token-causal mask.
+ *   - 3-D RoPE: d_rope is split into contiguous t, y, x segments of 2*rope_pairs[a]
+ *     elements; pair j of an axis segment with n pairs, elements (2j, 2j+1) of the
+ *     segment, is rotated by pos_a * rope_theta^(-j/n) radians.
+ *   - Accumulation is float32.  bfloat16 results are rounded to nearest even.
+ */
+#ifndef MLA_H
+#define MLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_ARG = 1,          /* null pointer, non-positive size, inconsistent shape      */
+  MLA_ERR_UNSUPPORTED = 2,  /* dtype or shape combination this library does not handle  */
+  MLA_ERR_ALIGN = 3,        /* a tensor pointer is not 16-byte aligned                  */
+  MLA_ERR_RANGE = 4,        /* token ranges outside the ring or the key window          */
+  MLA_ERR_CUDA = 5,         /* a CUDA launch failed                                     */
+  MLA_ERR_TIMEOUT = 6       /* a bounded device-side wait expired (see mla_device_error) */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+/* Problem shape.  64 bytes, no padding holes. */
+typedef struct {
+  int32_t batch;          /* B, independent sequences                                  */
+  int32_t n_heads;        /* n_h                                                       */
+  int32_t d_nope;         /* d_h, per-head content query/key/value width               */
+  int32_t d_latent;       /* d_c, shared content latent width                          */
+  int32_t d_rope;         /* d_R, shared decoupled RoPE key width (even)               */
+  int32_t rope_pairs[3];  /* rotation pairs on the t, y, x axes; sum = d_rope / 2      */
+  double  rope_theta;     /* RoPE base                                                  */
+  int32_t grid_h;         /* frame rows                                                 */
+  int32_t grid_w;         /* frame columns; tokens per frame F = grid_h * grid_w        */
+  int64_t ring_slots;     /* S, token slots per sequence in the ring                    */
+  int32_t dtype;          /* mla_dtype of every tensor argument                         */
+  int32_t reserved;       /* must be 0                                                   */
+} mla_shape;
+
+/*
+ * mla_cache_write — step 1: fused down-projection, 3-D RoPE and store into the ring.
+ * ("Multi-Head Latent Attention" concept page, "Low-rank joint compression": only
+ * the joint latent is cached; "The RoPE problem, and the decoupled fix": a small
+ * decoupled RoPE key is cached beside it, shared across heads.)
+ *
+ * For b < B and i < n_tok, with g = first_tok + i:
+ *   cache[b][g mod S][0 : d_latent]          = h[b][i] . w_dkv
+ *   cache[b][g mod S][d_latent : +d_rope]    = RoPE3D(h[b][i] . w_kr, position of g)
+ *   slots_out[b][i]                          = g mod S          (if slots_out != NULL)
+ *
+ *   h        [B, n_tok, d_model]                 storage dtype, read
+ *   w_dkv    [d_model, d_latent]                 storage dtype, read
+ *   w_kr     [d_model, d_rope]                   storage dtype, read
+ *   cache    [B, S, d_latent + d_rope]           storage dtype, written at n_tok slots
+ *   slots_out[B, n_tok] int32 or NULL            written
+ * Errors: MLA_ERR_RANGE if n_tok > S (a call may not overwrite its own rows) or
+ * first_tok < 0; MLA_ERR_ARG for null tensors or non-positive sizes.
+ */
+mla_status mla_cache_write(const mla_shape* shape, const void* h, int32_t d_model,
+                           int64_t n_tok, int64_t first_tok, const void* w_dkv,
+                           const void* w_kr, void* cache, int32_t* slots_out,
+                           void* stream);
+
+/*
+ * mla_absorb_q — step 2: query absorption through W_UK and RoPE of the query's
+ * decoupled part (concept page, "Low-rank joint compression": W^UK folds into the
+ * query side; "The RoPE problem, and the decoupled fix").
+ *
+ * For b, i < n_q, head h, with g = q_first_tok + i:
+ *   q_abs[b][i][h][0 : d_latent]       = q_nope[b][i][h] . w_uk[h]     ([d_nope] x [d_nope, d_latent])
+ *   q_abs[b][i][h][d_latent : +d_rope] = RoPE3D(q_rope[b][i][h], position of g)
+ *
+ *   q_nope [B, n_q, n_h, d_nope]           read
+ *   q_rope [B, n_q, n_h, d_rope]           read (un-rotated)
+ *   w_uk   [n_h, d_nope, d_latent]         read  (per-head key = w_uk[h] . c)
+ *   q_abs  [B, n_q, n_h, d_latent + d_rope] written
+ * Errors: MLA_ERR_ARG / MLA_ERR_RANGE (q_first_tok < 0).
+ */
+mla_status mla_absorb_q(const mla_shape* shape, const void* q_nope, const void* q_rope,
+                        int64_t n_q, int64_t q_first_tok, const void* w_uk, void* q_abs,
+                        void* stream);
+
+/*
+ * mla_attend_workspace_size — bytes of device workspace mla_attend needs for this
+ * problem (split-key partial results and their log-sum-exps).  May be 0.
+ */
+size_t mla_attend_workspace_size(const mla_shape* shape, int64_t n_q, int64_t n_keys);
+
+/*
+ * mla_attend — steps 3 and 4: absorbed attention in latent space over the ring
+ * (concept page, "Low-rank joint compression": one attends directly in latent space;
+ * "The RoPE problem, and the decoupled fix": score = content term + positional term;
+ * VideoMLA "The Gap": next-frame prediction over a sliding window).
+ *
+ * Keys are the global tokens k_first_tok .. k_first_tok + n_keys - 1, stored in slot
+ * g mod S.  Query i is token q_first_tok + i; it sees key g iff frame(g) <=
+ * frame(q) (frame-block-causal).  For every (b, i, h):
+ *   s(g)   = softmax_scale * (q_abs[b][i][h] . cache[b][g mod S])   (all d_latent+d_rope)
+ *   p      = softmax over the visible keys
+ *   o_lat[b][i][h] = sum_g p(g) * cache[b][g mod S][0 : d_latent]
+ *   lse[b][i][h]   = log(sum_g exp(s(g)))   (natural log, float32; if lse != NULL)
+ *
+ *   q_abs  [B, n_q, n_h, d_latent + d_rope]   read
+ *   cache  [B, S, d_latent + d_rope]          read
+ *   o_lat  [B, n_q, n_h, d_latent]            written
+ *   lse    [B, n_q, n_h] float32 or NULL      written
+ *   workspace: device scratch of at least mla_attend_workspace_size() bytes (may be
+ *   NULL when that size is 0); its contents on entry do not matter.
+ * A single query per sequence (n_q == 1) is the decode case.
+ * Errors: MLA_ERR_RANGE if n_keys > S, n_keys < 1, or the queries are not inside the
+ * key window (k_first_tok <= q_first_tok and q_first_tok + n_q <= k_first_tok +
+ * n_keys); MLA_ERR_ARG if workspace_bytes is too small.
+ */
+mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
+                      int64_t q_first_tok, const void* cache, int64_t k_first_tok,
+                      int64_t n_keys, float softmax_scale, void* o_lat, float* lse,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mla_up_v — step 5: per-head W_UV up-projection of the latent attention output
+ * (concept page, "Low-rank joint compression": W^UV is applied on the output side).
+ *   out[b][i][h] = w_uv[h] . o_lat[b][i][h]     ([d_nope, d_latent] x [d_latent])
+ *
+ *   o_lat [B, n_q, n_h, d_latent]   read
+ *   w_uv  [n_h, d_nope, d_latent]   read
+ *   out   [B, n_q, n_h, d_nope]     written
+ */
+mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q,
+                    const void* w_uv, void* out, void* stream);
+
+/*
+ * mla_kernel_launches — number of kernels this library has launched in this process
+ * (a host-side counter, incremented at every successful launch).  Diagnostic only.
+ */
+uint64_t mla_kernel_launches(void);
+
+/* Human-readable name of a status. Never NULL. */
+const char* mla_status_string(mla_status status);
+
+/*
+ * mla_device_error — synchronises `stream`, then reads and clears the library's
+ * device-side error word.  Returns MLA_ERR_TIMEOUT if a kernel gave up a bounded
+ * wait (on an mbarrier) since the last call, MLA_ERR_CUDA if the stream reports an
+ * error, else MLA_OK.  The only call that synchronises.
+ */
+mla_status mla_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H */

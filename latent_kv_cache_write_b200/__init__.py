@@ -1,0 +1,80 @@
+"""Absorbed multi-head latent attention over a sliding-window latent KV ring on B200.
+
+Python face of ``libmla.so``: the four calls of the C ABI under the same names, taking
+``torch`` CUDA tensors (or raw device pointers) and enqueuing on the current CUDA
+stream unless a stream is given.  PyTorch supplies device memory and streams only;
+all arithmetic runs in the library's kernels.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+from . import native
+from .native import MlaError, MlaShape, make_shape  # noqa: F401
+
+__all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
+           "mla_up_v", "mla_device_error", "mla_kernel_launches", "make_shape", "MlaShape", "MlaError"]
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def mla_cache_write(shape: MlaShape, h, d_model: int, n_tok: int, first_tok: int, w_dkv, w_kr,
+                    cache, slots_out=None, stream=None) -> None:
+    native.check("mla_cache_write", native.lib().mla_cache_write(
+        ctypes.byref(shape), _ptr(h), d_model, n_tok, first_tok, _ptr(w_dkv), _ptr(w_kr),
+        _ptr(cache), _ptr(slots_out), _stream(stream)))
+
+
+def mla_absorb_q(shape: MlaShape, q_nope, q_rope, n_q: int, q_first_tok: int, w_uk, q_abs,
+                 stream=None) -> None:
+    native.check("mla_absorb_q", native.lib().mla_absorb_q(
+        ctypes.byref(shape), _ptr(q_nope), _ptr(q_rope), n_q, q_first_tok, _ptr(w_uk),
+        _ptr(q_abs), _stream(stream)))
+
+
+def mla_attend_workspace_size(shape: MlaShape, n_q: int, n_keys: int) -> int:
+    return int(native.lib().mla_attend_workspace_size(ctypes.byref(shape), n_q, n_keys))
+
+
+def mla_attend(shape: MlaShape, q_abs, n_q: int, q_first_tok: int, cache, k_first_tok: int,
+               n_keys: int, softmax_scale: float, o_lat, lse=None, workspace=None,
+               workspace_bytes: Optional[int] = None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else (
+            workspace.numel() * workspace.element_size())
+    native.check("mla_attend", native.lib().mla_attend(
+        ctypes.byref(shape), _ptr(q_abs), n_q, q_first_tok, _ptr(cache), k_first_tok, n_keys,
+        softmax_scale, _ptr(o_lat), _ptr(lse), _ptr(workspace), workspace_bytes,
+        _stream(stream)))
+
+
+def mla_up_v(shape: MlaShape, o_lat, n_q: int, w_uv, out, stream=None) -> None:
+    native.check("mla_up_v", native.lib().mla_up_v(
+        ctypes.byref(shape), _ptr(o_lat), n_q, _ptr(w_uv), _ptr(out), _stream(stream)))
+
+
+def mla_kernel_launches() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(native.lib().mla_kernel_launches())
+
+
+def mla_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side error status."""
+    return int(native.lib().mla_device_error(_stream(stream)))

@@ -1,0 +1,47 @@
+// Internal launchers behind the C ABI (host side).  Each returns the CUDA error of its
+// launch.  Arguments have been validated by the ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+// Host-side count of kernels launched by the library (see mla_kernel_launches).
+void count_launches(int n);
+
+// SIMT CUDA-core path: every dtype and shape (float32 storage uses it throughout).
+cudaError_t simt_cache_write(const Geo& g, bool bf, const void* h, int d_model, int64_t n_tok,
+                             int64_t first_tok, const void* w_dkv, const void* w_kr,
+                             void* cache, int32_t* slots, cudaStream_t st);
+cudaError_t simt_absorb_q(const Geo& g, bool bf, const void* q_nope, const void* q_rope,
+                          int64_t n_q, int64_t q_first, const void* w_uk, void* q_abs,
+                          cudaStream_t st);
+cudaError_t simt_attend(const Geo& g, bool bf, const void* q_abs, int64_t n_q, int64_t q_first,
+                        const void* cache, int64_t k_first, int64_t n_keys, float scale,
+                        void* o_lat, float* lse, cudaStream_t st);
+cudaError_t simt_up_v(const Geo& g, bool bf, const void* o_lat, int64_t n_q, const void* w_uv,
+                      void* out, cudaStream_t st);
+
+// Tensor-core (tcgen05 + TMA) path for bf16 storage.
+bool tc_gemm_supported(const Geo& g, int d_model);
+cudaError_t tc_cache_write(const Geo& g, const void* h, int d_model, int64_t n_tok,
+                           int64_t first_tok, const void* w_dkv, const void* w_kr, void* cache,
+                           int32_t* slots, unsigned int* err, cudaStream_t st);
+cudaError_t tc_absorb_q(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,
+                        int64_t q_first, const void* w_uk, void* q_abs, unsigned int* err,
+                        cudaStream_t st);
+cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_uv, void* out,
+                    unsigned int* err, cudaStream_t st);
+
+bool tc_attend_supported(const Geo& g);
+cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
+                      const void* cache, int64_t k_first, int64_t n_keys, float scale,
+                      void* o_lat, float* lse, unsigned int* err, cudaStream_t st);
+
+// Device address of the library's error word on the current device (nullptr on failure).
+unsigned int* device_error_word();
+
+}  // namespace mla

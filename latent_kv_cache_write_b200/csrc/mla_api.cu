@@ -1,0 +1,195 @@
+// The C ABI: argument validation, then dispatch to the kernels.  Nothing is launched
+// unless every check passes.
+#include <stdio.h>
+
+#include <atomic>
+
+#include "launch.h"
+
+namespace mla {
+
+// Device-side error word; kernels that give up a bounded wait OR a code into it.
+__device__ unsigned int g_device_error = 0;
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+unsigned int* device_error_word() {
+  // One lookup per device: the symbol's address differs between devices.
+  static unsigned int* addr[64] = {};
+  static std::atomic<int> done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!done[dev].load(std::memory_order_acquire)) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+    done[dev].store(1, std::memory_order_release);
+  }
+  return addr[dev];
+}
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+mla_status check_shape(const mla_shape* s, Geo* g) {
+  if (!s) return MLA_ERR_ARG;
+  if (s->batch < 1 || s->n_heads < 1 || s->d_nope < 1 || s->d_latent < 1 || s->d_rope < 0)
+    return MLA_ERR_ARG;
+  if (s->grid_h < 1 || s->grid_w < 1 || s->ring_slots < 1 || s->reserved != 0)
+    return MLA_ERR_ARG;
+  if (s->d_rope % 2 != 0 || s->d_latent % 2 != 0) return MLA_ERR_ARG;
+  if (s->rope_pairs[0] < 0 || s->rope_pairs[1] < 0 || s->rope_pairs[2] < 0) return MLA_ERR_ARG;
+  if ((int64_t)s->rope_pairs[0] + s->rope_pairs[1] + s->rope_pairs[2] != s->d_rope / 2)
+    return MLA_ERR_ARG;
+  if (!(s->rope_theta > 0.0)) return MLA_ERR_ARG;
+  if (s->dtype != MLA_F32 && s->dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)s->d_latent + s->d_rope > 32 * 40) return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)s->batch * s->n_heads > 65535) return MLA_ERR_UNSUPPORTED;
+  g->B = s->batch; g->H = s->n_heads; g->Dn = s->d_nope; g->Dc = s->d_latent; g->Dr = s->d_rope;
+  for (int i = 0; i < 3; ++i) g->pairs[i] = s->rope_pairs[i];
+  g->theta = s->rope_theta;
+  g->gh = s->grid_h; g->gw = s->grid_w;
+  g->F = (int64_t)s->grid_h * s->grid_w;
+  g->S = s->ring_slots;
+  g->row = s->d_latent + s->d_rope;
+  return MLA_OK;
+}
+
+mla_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MLA_OK;
+  fprintf(stderr, "mla: CUDA error %s\n", cudaGetErrorString(e));
+  return MLA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_ARG: return "MLA_ERR_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_ALIGN: return "MLA_ERR_ALIGN";
+    case MLA_ERR_RANGE: return "MLA_ERR_RANGE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+mla_status mla_cache_write(const mla_shape* shape, const void* h, int32_t d_model,
+                           int64_t n_tok, int64_t first_tok, const void* w_dkv,
+                           const void* w_kr, void* cache, int32_t* slots_out, void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  if (d_model < 1 || n_tok < 0) return MLA_ERR_ARG;
+  if (!h || !w_dkv || !cache || (g.Dr > 0 && !w_kr)) return MLA_ERR_ARG;
+  if (first_tok < 0 || n_tok > g.S) return MLA_ERR_RANGE;
+  if (n_tok > INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(h) || !aligned16(w_dkv) || (w_kr && !aligned16(w_kr)) || !aligned16(cache) ||
+      (slots_out && !aligned16(slots_out)))
+    return MLA_ERR_ALIGN;
+  if (n_tok == 0) return MLA_OK;
+  const bool bf = shape->dtype == MLA_BF16;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (bf && g.Dr > 0 && tc_gemm_supported(g, d_model))
+    return cuda_status(tc_cache_write(g, h, d_model, n_tok, first_tok, w_dkv, w_kr, cache,
+                                      slots_out, device_error_word(), s));
+  return cuda_status(simt_cache_write(g, bf, h, d_model, n_tok, first_tok, w_dkv, w_kr, cache,
+                                      slots_out, s));
+}
+
+mla_status mla_absorb_q(const mla_shape* shape, const void* q_nope, const void* q_rope,
+                        int64_t n_q, int64_t q_first_tok, const void* w_uk, void* q_abs,
+                        void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  if (n_q < 0 || !q_nope || !w_uk || !q_abs || (g.Dr > 0 && !q_rope)) return MLA_ERR_ARG;
+  if (q_first_tok < 0) return MLA_ERR_RANGE;
+  if (n_q > INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_nope) || (q_rope && !aligned16(q_rope)) || !aligned16(w_uk) ||
+      !aligned16(q_abs))
+    return MLA_ERR_ALIGN;
+  if (n_q == 0) return MLA_OK;
+  const bool bf = shape->dtype == MLA_BF16;
+  if (bf && tc_gemm_supported(g, 0))
+    return cuda_status(tc_absorb_q(g, q_nope, q_rope, n_q, q_first_tok, w_uk, q_abs,
+                                   device_error_word(), (cudaStream_t)stream));
+  return cuda_status(simt_absorb_q(g, bf, q_nope, q_rope, n_q, q_first_tok, w_uk, q_abs,
+                                   (cudaStream_t)stream));
+}
+
+size_t mla_attend_workspace_size(const mla_shape* shape, int64_t n_q, int64_t n_keys) {
+  (void)shape; (void)n_q; (void)n_keys;
+  return 0;
+}
+
+mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
+                      int64_t q_first_tok, const void* cache, int64_t k_first_tok,
+                      int64_t n_keys, float softmax_scale, void* o_lat, float* lse,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  if (n_q < 0 || !q_abs || !cache || !o_lat) return MLA_ERR_ARG;
+  if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return MLA_ERR_ARG;
+  if (n_keys < 1 || n_keys > g.S || k_first_tok < 0 || q_first_tok < k_first_tok ||
+      q_first_tok + n_q > k_first_tok + n_keys)
+    return MLA_ERR_RANGE;
+  if (n_q > 65535) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(o_lat) || (lse && !aligned16(lse)))
+    return MLA_ERR_ALIGN;
+  const size_t need = mla_attend_workspace_size(shape, n_q, n_keys);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return MLA_ERR_ARG;
+  if (workspace && !aligned16(workspace)) return MLA_ERR_ALIGN;
+  if (n_q == 0) return MLA_OK;
+  const bool bf = shape->dtype == MLA_BF16;
+  if (bf && tc_attend_supported(g))
+    return cuda_status(tc_attend(g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                                 softmax_scale, o_lat, lse, device_error_word(),
+                                 (cudaStream_t)stream));
+  return cuda_status(simt_attend(g, bf, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                                 softmax_scale, o_lat, lse, (cudaStream_t)stream));
+}
+
+mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, const void* w_uv,
+                    void* out, void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  if (n_q < 0 || !o_lat || !w_uv || !out) return MLA_ERR_ARG;
+  if (n_q > INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(o_lat) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_ALIGN;
+  if (n_q == 0) return MLA_OK;
+  const bool bf = shape->dtype == MLA_BF16;
+  if (bf && tc_gemm_supported(g, 0))
+    return cuda_status(tc_up_v(g, o_lat, n_q, w_uv, out, device_error_word(),
+                               (cudaStream_t)stream));
+  return cuda_status(simt_up_v(g, bf, o_lat, n_q, w_uv, out, (cudaStream_t)stream));
+}
+
+uint64_t mla_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+mla_status mla_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  unsigned int word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (word != 0) {
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_status(e);
+    return MLA_ERR_TIMEOUT;
+  }
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,297 @@
+// Tensor-core (tcgen05) GEMMs of the path, bf16 in, fp32 accumulation in TMEM:
+//   cache write:  [h] x [W_DKV | W_KR]  -> RoPE on the W_KR columns -> bf16 -> ring slot
+//   absorb:       q_nope[:, h] x W_UK[h] -> q_lat (plus RoPE of q_R in the same CTAs)
+//   up-projection: o_lat[:, h] x W_UV[h]^T -> out
+// One 128 x BN output tile per CTA.  Warp 0 lane 0 issues TMA loads into a 4-stage
+// shared-memory ring, warp 1 lane 0 issues tcgen05.mma (M=128, N=BN, K=16 steps) into a
+// TMEM accumulator; afterwards all four warps read the accumulator (one row per
+// thread) and run the fused epilogue.
+#include "launch.h"
+#include "tc_ptx.cuh"
+#include "tmap.h"
+
+namespace mla {
+namespace {
+
+using namespace tc;
+
+constexpr int GBM = 128, GBK = 64, GSTAGES = 4, GBN = 128;
+constexpr int A_BYTES = GBM * GBK * 2;           // 16 KB
+constexpr int B_BYTES = GBN * GBK * 2;           // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int GEMM_SMEM = GSTAGES * STAGE_BYTES + 1024 + 256;
+
+enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
+
+struct TcGemm {
+  int M, N, K;
+  int mode;
+  int b_mn;                 // B is MN-major (N contiguous) instead of K-major
+  int n_split;              // cache: tiles at n >= n_split read tmB2 at n - n_split
+  bf16* out;
+  int64_t rows_per_batch;   // cache: tokens per sequence in the call (n_tok)
+  Geo geo;
+  int64_t first_tok;        // cache: first token; absorb: first query token
+  int32_t* slots;
+  const bf16* q_rope;       // absorb: RoPE part input
+  unsigned int* err;
+};
+
+__global__ void __launch_bounds__(128, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, TcGemm p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + GSTAGES * STAGE_BYTES);
+  uint64_t* empty = full + GSTAGES;
+  uint64_t* done = empty + GSTAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * GBM, n0 = blockIdx.y * GBN, z = blockIdx.z;
+  const bool second = p.mode == MODE_CACHE && n0 >= p.n_split;
+  const CUtensorMap* mB = second ? &tmB2 : &tmB;
+  const int nb = second ? n0 - p.n_split : n0;
+
+  if (tid == 0) {
+    for (int s = 0; s < GSTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(mB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, GBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = (p.K + GBK - 1) / GBK;
+
+  if (warp == 0 && lane == 0) {
+    // TMA producer
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % GSTAGES;
+      const uint32_t ph = (kb / GSTAGES) & 1;
+      if (!mbar_wait(&empty[s], ph ^ 1, abort, p.err)) break;
+      uint8_t* a = smem + s * STAGE_BYTES;
+      uint8_t* b = a + A_BYTES;
+      mbar_expect_tx(&full[s], STAGE_BYTES);
+      tma_load_3d(a, &tmA, &full[s], kb * GBK, p.mode == MODE_CACHE ? 0 : z, m0);
+      if (p.b_mn) {
+        tma_load_3d(b, mB, &full[s], nb, kb * GBK, z);
+        tma_load_3d(b + B_BYTES / 2, mB, &full[s], nb + 64, kb * GBK, z);
+      } else {
+        tma_load_3d(b, mB, &full[s], kb * GBK, nb, z);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    const uint32_t idesc = idesc_bf16(GBM, GBN, false, p.b_mn != 0);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % GSTAGES;
+      const uint32_t ph = (kb / GSTAGES) & 1;
+      if (!mbar_wait(&full[s], ph, abort, p.err)) break;
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
+      const uint32_t b = a + A_BYTES;
+      const uint64_t da = desc_sw128(a, 16, 1024);
+      const uint64_t db = p.b_mn ? desc_sw128(b, B_BYTES / 2, 1024) : desc_sw128(b, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < GBK / 16; ++ks) {
+        // K-major operands advance 32 bytes per 16-element K step inside the swizzle
+        // atom; the MN-major B advances 16 rows of 128 bytes.
+        const uint64_t bstep = p.b_mn ? (uint64_t)(ks * 2048 >> 4) : (uint64_t)(ks * 32 >> 4);
+        mma_ss(tmem, da + (uint64_t)(ks * 32 >> 4), db + bstep, idesc, (kb | ks) != 0);
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  // ---------------------------------------------------------------- epilogue
+  const bool ok = mbar_wait(done, 0, abort, p.err);
+  tc_fence_after();
+  const int r = warp * 32 + lane;
+  const int64_t m = m0 + r;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const Geo& G = p.geo;
+  for (int c0 = 0; c0 < GBN; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(trow + c0, v);
+    tmem_wait_ld();
+    if (!ok || m >= p.M) continue;
+    const int n = n0 + c0;                        // output column of v[0]
+    if (n >= p.N) continue;
+    float f[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+    bf16* dst;
+    if (p.mode == MODE_CACHE) {
+      const int64_t b = m / p.rows_per_batch;
+      const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
+      const int64_t slot = g % G.S;
+      if (n >= p.n_split) {
+#pragma unroll 4
+        for (int j = 0; j < 32; j += 2)
+          rope_rotate(f[j], f[j + 1], rope_angle(G, g, (n + j - p.n_split) / 2));
+      }
+      dst = p.out + (b * G.S + slot) * G.row + n;
+    } else if (p.mode == MODE_ABSORB) {
+      dst = p.out + (m * G.H + z) * G.row + n;
+    } else {
+      dst = p.out + (m * G.H + z) * G.Dn + n;
+    }
+    const int valid = p.N - n < 32 ? p.N - n : 32;
+    if (valid == 32) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16(f[8 * q + 0], f[8 * q + 1]);
+        w.y = pack_bf16(f[8 * q + 2], f[8 * q + 3]);
+        w.z = pack_bf16(f[8 * q + 4], f[8 * q + 5]);
+        w.w = pack_bf16(f[8 * q + 6], f[8 * q + 7]);
+        reinterpret_cast<uint4*>(dst)[q] = w;
+      }
+    } else {
+      for (int j = 0; j < valid; ++j) dst[j] = __float2bfloat16_rn(f[j]);
+    }
+  }
+  if (ok && m < p.M && blockIdx.y == 0) {
+    if (p.mode == MODE_CACHE && p.slots) {
+      const int64_t b = m / p.rows_per_batch;
+      const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
+      p.slots[m] = (int32_t)(g % G.S);
+    }
+    if (p.mode == MODE_ABSORB && G.Dr > 0) {
+      // q_abs[.., Dc:] = RoPE(q_R) for this CTA's rows and head
+      const int64_t i = m % p.rows_per_batch;
+      const int64_t g = p.first_tok + i;
+      const bf16* src = p.q_rope + (m * G.H + z) * G.Dr;
+      bf16* dst = p.out + (m * G.H + z) * G.row + G.Dc;
+      for (int q = 0; q < G.Dr / 2; ++q) {
+        float a = __bfloat162float(src[2 * q]), b = __bfloat162float(src[2 * q + 1]);
+        rope_rotate(a, b, rope_angle(G, g, q));
+        *reinterpret_cast<uint32_t*>(dst + 2 * q) = pack_bf16(a, b);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, GBN);
+  }
+}
+
+cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
+                   const TcGemm& p, int zcount, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((p.M + GBM - 1) / GBM, (p.N + GBN - 1) / GBN, zcount);
+  tc_gemm_kernel<<<grid, 128, GEMM_SMEM, st>>>(A, B, B2, p);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launches(1);
+  return e;
+}
+
+}  // namespace
+
+bool tc_gemm_supported(const Geo& g, int d_model) {
+  return g.Dc % GBN == 0 && g.Dr % 64 == 0 && g.Dn % 64 == 0 &&
+         (d_model <= 0 || d_model % 64 == 0);
+}
+
+cudaError_t tc_cache_write(const Geo& g, const void* h, int d_model, int64_t n_tok,
+                           int64_t first_tok, const void* w_dkv, const void* w_kr, void* cache,
+                           int32_t* slots, unsigned int* err, cudaStream_t st) {
+  CUtensorMap A, B, B2;
+  const uint64_t rows = (uint64_t)g.B * n_tok;
+  {
+    uint64_t d[3] = {(uint64_t)d_model, 1, rows};
+    uint64_t s[2] = {(uint64_t)d_model * 2, (uint64_t)d_model * 2};
+    uint32_t b[3] = {64, 1, 128};
+    if (!make_tmap_bf16(&A, h, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t d[3] = {(uint64_t)g.Dc, (uint64_t)d_model, 1};
+    uint64_t s[2] = {(uint64_t)g.Dc * 2, (uint64_t)g.Dc * d_model * 2};
+    uint32_t b[3] = {64, 64, 1};
+    if (!make_tmap_bf16(&B, w_dkv, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  if (g.Dr > 0) {
+    uint64_t d[3] = {(uint64_t)g.Dr, (uint64_t)d_model, 1};
+    uint64_t s[2] = {(uint64_t)g.Dr * 2, (uint64_t)g.Dr * d_model * 2};
+    uint32_t b[3] = {64, 64, 1};
+    if (!make_tmap_bf16(&B2, w_kr, 3, d, s, b)) return cudaErrorInvalidValue;
+  } else {
+    B2 = B;
+  }
+  TcGemm p{};
+  p.M = (int)rows; p.N = g.row; p.K = d_model; p.mode = MODE_CACHE; p.b_mn = 1;
+  p.n_split = g.Dc; p.out = (bf16*)cache; p.rows_per_batch = n_tok; p.geo = g;
+  p.first_tok = first_tok; p.slots = slots; p.err = err;
+  return launch(A, B, B2, p, 1, st);
+}
+
+cudaError_t tc_absorb_q(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,
+                        int64_t q_first, const void* w_uk, void* q_abs, unsigned int* err,
+                        cudaStream_t st) {
+  CUtensorMap A, B;
+  const uint64_t rows = (uint64_t)g.B * n_q;
+  {
+    uint64_t d[3] = {(uint64_t)g.Dn, (uint64_t)g.H, rows};
+    uint64_t s[2] = {(uint64_t)g.Dn * 2, (uint64_t)g.H * g.Dn * 2};
+    uint32_t b[3] = {64, 1, 128};
+    if (!make_tmap_bf16(&A, q_nope, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t d[3] = {(uint64_t)g.Dc, (uint64_t)g.Dn, (uint64_t)g.H};
+    uint64_t s[2] = {(uint64_t)g.Dc * 2, (uint64_t)g.Dc * g.Dn * 2};
+    uint32_t b[3] = {64, 64, 1};
+    if (!make_tmap_bf16(&B, w_uk, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  TcGemm p{};
+  p.M = (int)rows; p.N = g.Dc; p.K = g.Dn; p.mode = MODE_ABSORB; p.b_mn = 1;
+  p.n_split = 1 << 30; p.out = (bf16*)q_abs; p.rows_per_batch = n_q; p.geo = g;
+  p.first_tok = q_first; p.q_rope = (const bf16*)q_rope; p.err = err;
+  return launch(A, B, B, p, g.H, st);
+}
+
+cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_uv, void* out,
+                    unsigned int* err, cudaStream_t st) {
+  CUtensorMap A, B;
+  const uint64_t rows = (uint64_t)g.B * n_q;
+  {
+    uint64_t d[3] = {(uint64_t)g.Dc, (uint64_t)g.H, rows};
+    uint64_t s[2] = {(uint64_t)g.Dc * 2, (uint64_t)g.H * g.Dc * 2};
+    uint32_t b[3] = {64, 1, 128};
+    if (!make_tmap_bf16(&A, o_lat, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t d[3] = {(uint64_t)g.Dc, (uint64_t)g.Dn, (uint64_t)g.H};
+    uint64_t s[2] = {(uint64_t)g.Dc * 2, (uint64_t)g.Dc * g.Dn * 2};
+    uint32_t b[3] = {64, (uint32_t)GBN, 1};
+    if (!make_tmap_bf16(&B, w_uv, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  TcGemm p{};
+  p.M = (int)rows; p.N = g.Dn; p.K = g.Dc; p.mode = MODE_UPV; p.b_mn = 0;
+  p.n_split = 1 << 30; p.out = (bf16*)out; p.rows_per_batch = n_q; p.geo = g; p.err = err;
+  return launch(A, B, B, p, g.H, st);
+}
+
+}  // namespace mla

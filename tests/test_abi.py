@@ -1,0 +1,136 @@
+"""The C-ABI library loads, exports every symbol its header declares, and rejects bad
+arguments with the documented status before launching anything (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from latent_kv_cache_write_b200 import build, native
+from synth import configs as C
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "mla.h")
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: validation fails first
+ODD = 0x10008           # not 16-byte aligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return native.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:mla_status|size_t|uint64_t|const char\*)\s+(mla_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    syms = declared_symbols()
+    assert len(syms) >= 7, syms
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(syms) == set(native.SIGNATURES), "binding and header disagree"
+
+
+def test_shape_struct_layout():
+    assert ctypes.sizeof(native.MlaShape) == 64
+    assert native.MlaShape.rope_theta.offset == 32
+    assert native.MlaShape.ring_slots.offset == 48
+    text = open(HEADER).read()
+    assert "64 bytes, no padding holes" in text
+
+
+def test_status_strings(L):
+    for code, name in enumerate(["MLA_OK", "MLA_ERR_ARG", "MLA_ERR_UNSUPPORTED", "MLA_ERR_ALIGN",
+                                 "MLA_ERR_RANGE", "MLA_ERR_CUDA", "MLA_ERR_TIMEOUT"]):
+        assert native.status_string(code) == name
+    assert native.status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def _shape(**kw):
+    s = native.make_shape(C.VIDEO_CHUNK)
+    for k, v in kw.items():
+        if k == "rope_pairs":
+            s.rope_pairs[:] = v
+        else:
+            setattr(s, k, v)
+    return s
+
+
+def _attend(L, s, q=FAKE, n_q=1560, q_first=3 * 1560, cache=FAKE, k_first=0, n_keys=6240,
+            scale=0.07, o=FAKE, lse=None, ws=None, ws_bytes=0):
+    return L.mla_attend(ctypes.byref(s), q, n_q, q_first, cache, k_first, n_keys, scale, o, lse,
+                        ws, ws_bytes, None)
+
+
+def test_shape_validation(L):
+    bad = [dict(batch=0), dict(n_heads=0), dict(d_rope=63), dict(rope_pairs=[8, 12, 11]),
+           dict(rope_pairs=[-1, 21, 12]), dict(grid_h=0), dict(ring_slots=0), dict(reserved=1),
+           dict(rope_theta=0.0), dict(d_latent=511)]
+    for kw in bad:
+        assert _attend(L, _shape(**kw)) == native.MLA_ERR_ARG, kw
+    assert _attend(L, _shape(dtype=7)) == native.MLA_ERR_UNSUPPORTED
+    assert L.mla_attend(None, FAKE, 1, 0, FAKE, 0, 1, 1.0, FAKE, None, None, 0, None) == \
+        native.MLA_ERR_ARG
+
+
+def test_attend_ranges_and_pointers(L):
+    s = _shape()
+    R = native.MLA_ERR_RANGE
+    assert _attend(L, s, n_keys=6241) == R                    # more keys than ring slots
+    assert _attend(L, s, n_keys=0) == R
+    assert _attend(L, s, k_first=-1) == R
+    assert _attend(L, s, q_first=0, k_first=1) == R            # query before the window
+    assert _attend(L, s, q_first=3 * 1560 + 1) == R            # query past the window
+    assert _attend(L, s, q=None) == native.MLA_ERR_ARG
+    assert _attend(L, s, cache=None) == native.MLA_ERR_ARG
+    assert _attend(L, s, o=None) == native.MLA_ERR_ARG
+    assert _attend(L, s, scale=0.0) == native.MLA_ERR_ARG
+    assert _attend(L, s, scale=float("nan")) == native.MLA_ERR_ARG
+    assert _attend(L, s, q=ODD) == native.MLA_ERR_ALIGN
+    assert _attend(L, s, lse=ODD) == native.MLA_ERR_ALIGN
+    assert _attend(L, s, n_q=-1) == native.MLA_ERR_ARG
+
+
+def test_attend_workspace_check(L):
+    s = _shape()
+    need = L.mla_attend_workspace_size(ctypes.byref(s), 1560, 6240)
+    if need:
+        assert _attend(L, s, ws=FAKE, ws_bytes=need - 1) == native.MLA_ERR_ARG
+        assert _attend(L, s, ws=None, ws_bytes=need) == native.MLA_ERR_ARG
+
+
+def test_cache_write_validation(L):
+    s = _shape()
+    cw = lambda **k: L.mla_cache_write(
+        ctypes.byref(s), k.get("h", FAKE), k.get("d", 4096), k.get("n", 1560),
+        k.get("first", 0), k.get("wd", FAKE), k.get("wr", FAKE), k.get("cache", FAKE),
+        k.get("slots", None), None)
+    assert cw(n=6241) == native.MLA_ERR_RANGE
+    assert cw(first=-1) == native.MLA_ERR_RANGE
+    assert cw(d=0) == native.MLA_ERR_ARG
+    assert cw(h=None) == native.MLA_ERR_ARG
+    assert cw(wr=None) == native.MLA_ERR_ARG
+    assert cw(cache=ODD) == native.MLA_ERR_ALIGN
+    assert cw(slots=ODD) == native.MLA_ERR_ALIGN
+    assert cw(n=0) == native.MLA_OK                             # empty: nothing to do
+
+
+def test_absorb_and_up_v_validation(L):
+    s = _shape()
+    ab = lambda **k: L.mla_absorb_q(ctypes.byref(s), k.get("qn", FAKE), k.get("qr", FAKE),
+                                    k.get("n", 1560), k.get("first", 0), k.get("w", FAKE),
+                                    k.get("out", FAKE), None)
+    assert ab(first=-1) == native.MLA_ERR_RANGE
+    assert ab(qn=None) == native.MLA_ERR_ARG
+    assert ab(out=ODD) == native.MLA_ERR_ALIGN
+    assert ab(n=0) == native.MLA_OK
+    uv = lambda **k: L.mla_up_v(ctypes.byref(s), k.get("o", FAKE), k.get("n", 1560),
+                                k.get("w", FAKE), k.get("out", FAKE), None)
+    assert uv(o=None) == native.MLA_ERR_ARG
+    assert uv(w=ODD) == native.MLA_ERR_ALIGN
+    assert uv(n=-2) == native.MLA_ERR_ARG
+    assert uv(n=0) == native.MLA_OK

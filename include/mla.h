@@ -182,6 +182,13 @@ const char* mla_status_string(mla_status status);
  */
 mla_status mla_device_error(void* stream);
 
+/*
+ * mla_device_error_info — details of the last device-side error that mla_device_error
+ * reported: info[0] status bits, info[1] id of the first wait site that gave up,
+ * info[2] its CTA index, info[3] a (thread << 16 | block) tag.  Zeros if none yet.
+ */
+void mla_device_error_info(uint32_t info[4]);
+
 #ifdef __cplusplus
 }
 #endif

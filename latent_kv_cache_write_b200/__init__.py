@@ -15,7 +15,7 @@ from . import native
 from .native import MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
-           "mla_up_v", "mla_device_error", "mla_kernel_launches", "make_shape", "MlaShape", "MlaError"]
+           "mla_up_v", "mla_device_error", "mla_kernel_launches", "mla_device_error_info", "make_shape", "MlaShape", "MlaError"]
 
 
 def _ptr(t) -> Optional[int]:
@@ -73,6 +73,14 @@ def mla_up_v(shape: MlaShape, o_lat, n_q: int, w_uv, out, stream=None) -> None:
 def mla_kernel_launches() -> int:
     """Kernels launched by the library so far in this process."""
     return int(native.lib().mla_kernel_launches())
+
+
+def mla_device_error_info() -> list:
+    """[status bits, wait site id, CTA index, (thread << 16 | block)] of the last
+    device-side error reported by mla_device_error."""
+    buf = (ctypes.c_uint32 * 4)()
+    native.lib().mla_device_error_info(buf)
+    return list(buf)
 
 
 def mla_device_error(stream=None) -> int:

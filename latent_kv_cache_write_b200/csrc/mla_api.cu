@@ -8,8 +8,10 @@
 
 namespace mla {
 
-// Device-side error word; kernels that give up a bounded wait OR a code into it.
-__device__ unsigned int g_device_error = 0;
+// Device-side error words: [0] status bits ORed by a kernel that gave up a bounded wait,
+// [1] site id of the first such wait, [2] its CTA index, [3] its (thread, block) tag.
+__device__ unsigned int g_device_error[4] = {0, 0, 0, 0};
+static unsigned int g_last_error_info[4] = {0, 0, 0, 0};
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -176,16 +178,21 @@ mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, cons
   return cuda_status(simt_up_v(g, bf, o_lat, n_q, w_uv, out, (cudaStream_t)stream));
 }
 
+void mla_device_error_info(uint32_t info[4]) {
+  for (int i = 0; i < 4; ++i) info[i] = g_last_error_info[i];
+}
+
 uint64_t mla_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 mla_status mla_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e);
-  unsigned int word = 0, zero = 0;
-  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+  unsigned int words[4] = {0, 0, 0, 0}, zero[4] = {0, 0, 0, 0};
+  e = cudaMemcpyFromSymbol(words, g_device_error, sizeof(words));
   if (e != cudaSuccess) return cuda_status(e);
-  if (word != 0) {
-    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (words[0] != 0) {
+    for (int i = 0; i < 4; ++i) g_last_error_info[i] = words[i];
+    e = cudaMemcpyToSymbol(g_device_error, zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_status(e);
     return MLA_ERR_TIMEOUT;
   }

@@ -69,6 +69,7 @@ constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int ATT_SMEM = OFF_MISC + 16 + 1024;
 
 constexpr uint32_t O_COL = 0, Q_COL = 256, S_COL = 384;
+constexpr unsigned FULL = 0xffffffffu;
 
 struct AttnArgs {
   Geo g;
@@ -194,7 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const uint32_t bytes = rank == 1 ? STAGE_BYTES : LAT_BYTES;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NST;
-        if (!mbar_wait(&bar[B_KVE + s], ((j / NST) & 1) ^ 1, abort, a.err)) break;
+        if (!mbar_wait(&bar[B_KVE + s], ((j / NST) & 1) ^ 1, abort, a.err, 0x101, j)) break;
         int64_t slot0, g0;
         int valid;
         blk.get(j, slot0, g0, valid);
@@ -213,12 +214,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, BN, false, false);
       const uint32_t id_pv = idesc_bf16(128, HALF, false, true);
-      bool ok = mbar_wait(&bar[B_QREADY], 0, abort, a.err);
-      if (ok && rank == 1) ok = mbar_wait(&bar[B_QR], 0, abort, a.err);
+      bool ok = mbar_wait(&bar[B_QREADY], 0, abort, a.err, 0x102, 0);
+      if (ok && rank == 1) ok = mbar_wait(&bar[B_QR], 0, abort, a.err, 0x103, 0);
       tc_fence_after();
       auto pv = [&](int jj) -> bool {
         const int pb = jj & 1;
-        if (!mbar_wait(&bar[B_PF + pb], (jj >> 1) & 1, abort, a.err)) return false;
+        if (!mbar_wait(&bar[B_PF + pb], (jj >> 1) & 1, abort, a.err, 0x104, jj)) return false;
         tc_fence_after();
         const uint32_t st = smem_u32(sm + OFF_KV + (jj % NST) * STAGE_BYTES);
         const uint32_t pa = smem_u32(sm + OFF_P + pb * P_BYTES);
@@ -232,8 +233,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       };
       for (int j = 0; ok && j < nblk; ++j) {
         const int s = j % NST, sb = j & 1;
-        if (!mbar_wait(&bar[B_KVF + s], (j / NST) & 1, abort, a.err)) break;
-        if (!mbar_wait(&bar[B_SE + sb], ((j >> 1) & 1) ^ 1, abort, a.err)) break;
+        if (!mbar_wait(&bar[B_KVF + s], (j / NST) & 1, abort, a.err, 0x105, j)) break;
+        if (!mbar_wait(&bar[B_SE + sb], ((j >> 1) & 1) ^ 1, abort, a.err, 0x106, j)) break;
         tc_fence_after();
         const uint32_t d = tmem + S_COL + sb * BN;
         const uint32_t st = smem_u32(sm + OFF_KV + s * STAGE_BYTES);
@@ -290,7 +291,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     for (int j = 0; j < nblk; ++j) {
       const int sb = j & 1;
       const uint32_t kph = (j >> 1) & 1;
-      if (!mbar_wait(&bar[B_SF + sb], kph, abort, a.err)) { ok = false; break; }
+      if (!__all_sync(FULL, mbar_wait(&bar[B_SF + sb], kph, abort, a.err, 0x201, (t << 16) | j))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       float s[64];
       {
@@ -312,7 +316,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
       if (!owner) {
         // partial scores of the peer's rows -> peer's exchange buffer
-        if (!mbar_wait_cluster(&bar[B_XE + sb], kph ^ 1, abort, a.err)) { ok = false; break; }
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + sb], kph ^ 1, abort, a.err, 0x202,
+                                                 (t << 16) | j))) {
+          ok = false;
+          break;
+        }
         const uint32_t dst = mapa(smem_u32(sm + OFF_X + sb * X_BYTES), peer) +
                              (uint32_t)(t - (int)peer * 64) * (BN * 4);
 #pragma unroll
@@ -324,7 +332,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         // keys contribute exact zeros to P.V whatever the ring holds there
         if (valid < BN) {
           const int s_idx = j % NST;
-          if (!mbar_wait(&bar[B_KVF + s_idx], (j / NST) & 1, abort, a.err)) { ok = false; break; }
+          if (!__all_sync(FULL, mbar_wait(&bar[B_KVF + s_idx], (j / NST) & 1, abort, a.err, 0x203,
+                                          (t << 16) | j))) {
+            ok = false;
+            break;
+          }
           const int u = t - (int)peer * 64;               // 0..63
           if (u >= valid) {
             uint8_t* st = sm + OFF_KV + s_idx * STAGE_BYTES + u * 128;
@@ -337,15 +349,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           }
         }
         // this row's P and rescale factor from the owner
-        if (!mbar_wait_cluster(&bar[B_RF + sb], kph, abort, a.err)) { ok = false; break; }
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_RF + sb], kph, abort, a.err, 0x204,
+                                                 (t << 16) | j))) {
+          ok = false;
+          break;
+        }
         const float fac = F[sb * TM + t];
         if (j > 0) {
-          if (!mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort, a.err)) {
+          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
+                                          a.err, 0x205, (t << 16) | j))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (fac != 1.f) rescale_row(tmem + lane_base + O_COL, fac);
+          // warp-collective TMEM access: every lane runs it, factor 1 where nothing grew
+          if (__any_sync(FULL, fac != 1.f)) rescale_row(tmem + lane_base + O_COL, fac);
           // my P buffer of block j-1 is free again: the peer may write block j+1 rows
           mbar_arrive_cluster(peer_bar(B_PPE + ((j - 1) & 1)));
         }
@@ -354,7 +372,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         mbar_arrive(&bar[B_PF + sb]);
       } else {
         // full scores: add the peer's partial
-        if (!mbar_wait_cluster(&bar[B_XF + sb], kph, abort, a.err)) { ok = false; break; }
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + sb], kph, abort, a.err, 0x301,
+                                                 (t << 16) | j))) {
+          ok = false;
+          break;
+        }
         const float4* xr = reinterpret_cast<const float4*>(sm + OFF_X + sb * X_BYTES +
                                                            (t - (int)rank * 64) * (BN * 4));
 #pragma unroll
@@ -387,17 +409,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           pk[c] = pack_bf16(p0, p1);
         }
         l = l * fac + sum;
-        if (j > 0 && fac != 1.f) {
-          if (!mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort, a.err)) {
+        // warp-collective TMEM access: the whole warp rescales if any of its rows grew
+        if (j > 0 && __any_sync(FULL, fac != 1.f)) {
+          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
+                                          a.err, 0x302, (t << 16) | j))) {
             ok = false;
             break;
           }
           tc_fence_after();
           rescale_row(tmem + lane_base + O_COL, fac);
         } else if (j >= 2) {
-          if (!mbar_wait(&bar[B_PE + sb], kph ^ 1, abort, a.err)) { ok = false; break; }
+          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + sb], kph ^ 1, abort, a.err, 0x303,
+                                          (t << 16) | j))) {
+            ok = false;
+            break;
+          }
         }
-        if (!mbar_wait_cluster(&bar[B_PPE + sb], kph ^ 1, abort, a.err)) { ok = false; break; }
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_PPE + sb], kph ^ 1, abort, a.err, 0x304,
+                                                 (t << 16) | j))) {
+          ok = false;
+          break;
+        }
         uint8_t* prow = sm + OFF_P + sb * P_BYTES + t * 128;
         const uint32_t prem = mapa(smem_u32(prow), peer);
 #pragma unroll
@@ -417,7 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = mbar_wait(&bar[B_DONE], 0, abort, a.err);
+    if (ok) ok = mbar_wait(&bar[B_DONE], 0, abort, a.err, 0x401, t);
     tc_fence_after();
     float inv = 0.f;
     if (owner) {
@@ -426,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_arrive_cluster(peer_bar(B_FIN));
       if (a.lse && row_valid && ok) a.lse[grow] = (m + log2f(l)) * 0.69314718055994530942f;
     } else {
-      if (ok) ok = mbar_wait_cluster(&bar[B_FIN], 0, abort, a.err);
+      if (ok) ok = mbar_wait_cluster(&bar[B_FIN], 0, abort, a.err, 0x402, t);
       inv = F[2 * TM + t];
     }
     bf16* dst = a.o_lat + grow * G.Dc + rank * HALF;
@@ -450,8 +482,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 
   // ------------------------------------------------------------ teardown
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
   cluster_sync();          // no remote access into this CTA is still pending
   if (warp == 5) {
     tc_fence_after();

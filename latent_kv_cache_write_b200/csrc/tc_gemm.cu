@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(128, 1)
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % GSTAGES;
       const uint32_t ph = (kb / GSTAGES) & 1;
-      if (!mbar_wait(&empty[s], ph ^ 1, abort, p.err)) break;
+      if (!mbar_wait(&empty[s], ph ^ 1, abort, p.err, 0x11, kb)) break;
       uint8_t* a = smem + s * STAGE_BYTES;
       uint8_t* b = a + A_BYTES;
       mbar_expect_tx(&full[s], STAGE_BYTES);
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(128, 1)
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % GSTAGES;
       const uint32_t ph = (kb / GSTAGES) & 1;
-      if (!mbar_wait(&full[s], ph, abort, p.err)) break;
+      if (!mbar_wait(&full[s], ph, abort, p.err, 0x12, kb)) break;
       tc_fence_after();
       const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
       const uint32_t b = a + A_BYTES;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncwarp();
 
   // ---------------------------------------------------------------- epilogue
-  const bool ok = mbar_wait(done, 0, abort, p.err);
+  const bool ok = mbar_wait(done, 0, abort, p.err, 0x13, tid);
   tc_fence_after();
   const int r = warp * 32 + lane;
   const int64_t m = m0 + r;

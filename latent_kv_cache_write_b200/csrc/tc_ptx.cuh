@@ -78,44 +78,53 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Record a timed-out wait in the library's error word array err[0..3]: err[0] |= 1;
+// the first timeout also stores its site id, CTA index and (thread, block) tag.
+__device__ __forceinline__ void report_timeout(unsigned int* err, uint32_t site, uint32_t tag) {
+  if (!err) return;
+  atomicOr(err, 1u);
+  if (atomicCAS(err + 1, 0u, site) == 0u) {
+    err[2] = blockIdx.x;
+    err[3] = tag;
+  }
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after ~2 s of wall
-// time (a wait that long means a bug, not a slow pipeline): sets *abort, ORs the
-// timeout code into the device error word and returns false.  Returns false at once
-// if *abort is already set by another thread of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+// time (a wait that long means a bug, not a slow pipeline): sets *abort, reports the
+// site and returns false.  Returns false at once if *abort is already set by another
+// thread of the CTA.  ACQ_CLUSTER selects cluster-scope acquire, for barriers that the
+// peer CTA of a cluster arrives on after writing into this CTA's shared memory.
+template <bool ACQ_CLUSTER>
+__device__ __forceinline__ bool mbar_wait_t(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            unsigned int* err, uint32_t site, uint32_t tag) {
+  auto probe = [&]() {
+    return ACQ_CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (probe()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (probe()) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > 2000000000ull) {
         *abort = 1;
-        if (err) atomicOr(err, 1u);
+        report_timeout(err, site, tag);
         return false;
       }
     }
   }
 }
 
-// Same as mbar_wait, with cluster-scope acquire: for barriers that the peer CTA of the
-// cluster arrives on after writing into this CTA's shared memory.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned int* err, uint32_t site = 0xFFu,
+                                          uint32_t tag = 0) {
+  return mbar_wait_t<false>(bar, parity, abort, err, site, tag);
+}
+
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, unsigned int* err) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
-        *abort = 1;
-        if (err) atomicOr(err, 1u);
-        return false;
-      }
-    }
-  }
+                                                  volatile int* abort, unsigned int* err,
+                                                  uint32_t site = 0xFFu, uint32_t tag = 0) {
+  return mbar_wait_t<true>(bar, parity, abort, err, site, tag);
 }
 
 // ------------------------------------------------------------------ clusters / DSMEM

@@ -23,7 +23,7 @@ def L():
 
 def declared_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:mla_status|size_t|uint64_t|const char\*)\s+(mla_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:mla_status|size_t|uint64_t|void|const char\*)\s+(mla_\w+)\s*\(",
                                  text, re.M)))
 
 

@@ -11,16 +11,23 @@
 //   - TMA-loads its columns of the 64 cached rows (one load serves as K and as V),
 //   - computes its partial score S_c = Q_c . K_c^T with tcgen05.mma (Q's latent half
 //     resident in TMEM as the A operand, the RoPE part from shared memory),
-//   - exchanges partial scores through distributed shared memory: CTA c finishes the
-//     softmax of rows [64c, 64c + 64) and receives the peer's partials for them,
-//   - writes its P rows (bf16) into both CTAs' shared memory with the rescale factors,
+//   - swaps partial scores with its peer through distributed shared memory, so both
+//     CTAs hold the full scores of all 128 rows,
+//   - runs the online softmax of all 128 rows itself (both CTAs take bit-identical
+//     decisions: the same fp32 sums in the same order),
 //   - accumulates O_c += P . V_c (M=128, N=256) into its TMEM.
-// The online softmax keeps a running max per row and rescales O only when the max grows
-// by more than 8 (log2 units).  Masking is frame-block-causal per row; a ring that
-// wraps is walked as two contiguous slot segments.
 //
-// Warp roles (192 threads): warps 0-3 softmax / exchange / epilogue (thread = row =
-// TMEM lane), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner.
+// Two softmax warpgroups take alternate key blocks, so the exchange of one block
+// overlaps the exponentials of the other; they hand the running row maximum to each
+// other through shared memory.  P (bf16) is written over the block's consumed exchange
+// buffer; the peer may refill that buffer once the PV product reading it has finished,
+// which the MMA thread signals straight into the peer's barrier with a multicast
+// tcgen05.commit.  O is rescaled only when a row maximum grows by more than 8 (log2
+// units).  Masking is frame-block-causal per row; a ring that wraps is walked as two
+// contiguous slot segments.
+//
+// Warp roles (320 threads): warps 0-3 and 4-7 are the two softmax warpgroups (thread =
+// row = TMEM lane), warp 8 is the TMA producer, warp 9 the MMA issuer and TMEM owner.
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tmap.h"
@@ -38,31 +45,32 @@ constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
 constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB
 constexpr int STAGE_BYTES = LAT_BYTES + BOX_BYTES;    // + RoPE box (CTA 1)
 constexpr int QR_BYTES = TM * 64 * 2;                 // Q RoPE part, 16 KB
-constexpr int P_BYTES = TM * BN * 2;                  // 16 KB
-constexpr int X_BYTES = 64 * BN * 4;                  // 16 KB
+constexpr int X_BYTES = TM * BN * 4;                  // exchange buffer, 32 KB: the peer's
+                                                      // partial scores, chunk-major
+                                                      // [16 x float4][128 rows]; then P
+                                                      // (bf16, 128-byte swizzled rows)
+constexpr int NTHREADS = 320;
 
 constexpr int OFF_KV = 0;
 constexpr int OFF_QR = OFF_KV + NST * STAGE_BYTES;
-constexpr int OFF_P = OFF_QR + QR_BYTES;
-constexpr int OFF_X = OFF_P + 2 * P_BYTES;
-constexpr int OFF_F = OFF_X + 2 * X_BYTES;            // factors [2][128] + final 1/l [128]
-constexpr int OFF_BAR = OFF_F + 3 * TM * 4;
+constexpr int OFF_X = OFF_QR + QR_BYTES;              // [2] exchange / P buffers
+constexpr int OFF_M = OFF_X + 2 * X_BYTES;            // running max handoff [2][128]
+constexpr int OFF_L = OFF_M + 2 * TM * 4;             // final (l, m) per warpgroup [2][2][128]
+constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
 
 enum {
   B_KVF = 0,                // K/V stage loaded (TMA)
   B_KVE = B_KVF + NST,      // K/V stage free (MMA commit after PV)
   B_QR = B_KVE + NST,       // Q RoPE tile loaded
-  B_QREADY,                 // Q latent half written to TMEM (128 threads)
-  B_SF,                     // S buffer full (MMA commit)          [2]
-  B_SE = B_SF + 2,          // S buffer read (128 threads)         [2]
-  B_XF = B_SE + 2,          // peer partials landed in my X        [2] 64 remote
-  B_XE = B_XF + 2,          // peer consumed my partials           [2] 64 remote
-  B_RF = B_XE + 2,          // peer P rows + factors landed        [2] 64 remote
-  B_PF = B_RF + 2,          // P buffer complete, O rescaled       [2] 128
-  B_PE = B_PF + 2,          // PV done with P buffer               [2] commit
-  B_PPE = B_PE + 2,         // peer's P buffer free for my rows    [2] 64 remote
-  B_FIN = B_PPE + 2,        // peer's final 1/l landed                 64 remote
-  B_DONE,                   // every MMA finished
+  B_QREADY,                 // Q latent half written to TMEM (256 threads)
+  B_SF,                     // S buffer full (MMA commit)                  [2]
+  B_SE = B_SF + 2,          // S buffer read (128 threads)                 [2]
+  B_XF = B_SE + 2,          // peer's partial scores landed (tx bytes)     [2]
+  B_XE = B_XF + 2,          // peer's PV done with its buffer (1 remote)   [2]
+  B_PF = B_XE + 2,          // P complete, O rescaled (128)                [2]
+  B_PE = B_PF + 2,          // PV done (MMA commit)                        [2]
+  B_M = B_PE + 2,           // running max of a block published (128)      [2]
+  B_DONE = B_M + 2,         // every MMA finished
   NBAR
 };
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -115,7 +123,7 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                   AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -124,7 +132,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
-  float* F = reinterpret_cast<float*>(sm + OFF_F);
 
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -158,23 +165,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(&bar[B_KVE + s], 1);
     }
     mbar_init(&bar[B_QR], 1);
-    mbar_init(&bar[B_QREADY], 128);
+    mbar_init(&bar[B_QREADY], 256);
     for (int q = 0; q < 2; ++q) {
       mbar_init(&bar[B_SF + q], 1);
       mbar_init(&bar[B_SE + q], 128);
-      mbar_init(&bar[B_XF + q], 64);
-      mbar_init(&bar[B_XE + q], 64);
-      mbar_init(&bar[B_RF + q], 64);
+      mbar_init(&bar[B_XF + q], 1);
+      mbar_init(&bar[B_XE + q], 1);
       mbar_init(&bar[B_PF + q], 128);
       mbar_init(&bar[B_PE + q], 1);
-      mbar_init(&bar[B_PPE + q], 64);
+      mbar_init(&bar[B_M + q], 128);
     }
-    mbar_init(&bar[B_FIN], 64);
     mbar_init(&bar[B_DONE], 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -183,7 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
@@ -209,7 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           tma_load_3d(st + LAT_BYTES, &tmK, &bar[B_KVF + s], G.Dc, (int32_t)slot0, b);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, BN, false, false);
@@ -222,13 +227,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (!mbar_wait(&bar[B_PF + pb], (jj >> 1) & 1, abort, a.err, 0x104, jj)) return false;
         tc_fence_after();
         const uint32_t st = smem_u32(sm + OFF_KV + (jj % NST) * STAGE_BYTES);
-        const uint32_t pa = smem_u32(sm + OFF_P + pb * P_BYTES);
+        const uint32_t pa = smem_u32(sm + OFF_X + pb * X_BYTES);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
                  desc_sw128(st + ks * 2048, BOX_BYTES, 1024), id_pv, (jj > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bar[B_PE + pb]);
         mma_commit(&bar[B_KVE + jj % NST]);
+        // the peer's warpgroup waits for this before refilling the buffer at block jj+2;
+        // no signal is sent that nobody waits for (the peer may have exited by then)
+        if (jj + 2 < nblk) mma_commit_cluster(&bar[B_XE + pb], (uint16_t)(1u << peer));
         return true;
       };
       for (int j = 0; ok && j < nblk; ++j) {
@@ -257,41 +265,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mma_commit(&bar[B_DONE]);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int t = tid;                         // row of the tile == TMEM lane
-    const bool owner = (uint32_t)(t >> 6) == rank;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;                  // warpgroup: even (0) or odd (1) blocks
+    const int t = tid & (TM - 1);              // row of the tile == TMEM lane
     const int64_t r_in_b = row0 + t;
     const bool row_valid = r_in_b < rows_b;
     const int64_t grow = grow0 + t;
     const int64_t k_end_row = k_end_of(row_valid ? r_in_b / G.H : i_last);
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t peer_bar0 = mapa(smem_u32(bar), peer);
-    auto peer_bar = [&](int idx) { return peer_bar0 + idx * 8; };
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    float* m_sh = reinterpret_cast<float*>(sm + OFF_M);
+    float* l_sh = reinterpret_cast<float*>(sm + OFF_L);
 
-    // Q latent half -> TMEM (A operand of the score MMA), bf16 pairs per column
+    // Q latent half -> TMEM (A operand of the score MMA), bf16 pairs per column; each
+    // warpgroup loads half of the row
     {
-      const uint4* src = reinterpret_cast<const uint4*>(a.q_abs + grow * G.row + rank * HALF);
+      const uint4* src = reinterpret_cast<const uint4*>(a.q_abs + grow * G.row + rank * HALF +
+                                                        wg * (HALF / 2));
 #pragma unroll 1
-      for (int c = 0; c < HALF / 32; ++c) {
+      for (int c = 0; c < HALF / 64; ++c) {
         uint32_t v[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 x = row_valid ? src[c * 4 + q] : make_uint4(0, 0, 0, 0);
           v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
         }
-        tmem_st16(tmem + lane_base + Q_COL + c * 16, v);
+        tmem_st16(tmem + lane_base + Q_COL + wg * (HALF / 4) + c * 16, v);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar[B_QREADY]);
     }
 
-    float m = -INFINITY, l = 0.f;
+    const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * X_BYTES), peer) + (uint32_t)t * 16;
+    const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
+    const float4* my_x = reinterpret_cast<const float4*>(sm + OFF_X + wg * X_BYTES) + t;
+    uint8_t* prow = sm + OFF_X + wg * X_BYTES + t * 128;     // P row t over the same buffer
+    const float c2 = a.scale_log2;
+    float m_last = -INFINITY, l = 0.f;         // this warpgroup's running sum and its max
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
-      const int sb = j & 1;
+    for (int j = wg; j < nblk; j += 2) {
       const uint32_t kph = (j >> 1) & 1;
-      if (!__all_sync(FULL, mbar_wait(&bar[B_SF + sb], kph, abort, a.err, 0x201, (t << 16) | j))) {
+      // arm this block's exchange: the peer's asynchronous stores complete X_BYTES of
+      // transactions on it (they may land before or after this arrive)
+      if (t == 0) mbar_expect_tx(&bar[B_XF + wg], X_BYTES);
+      if (!__all_sync(FULL, mbar_wait(&bar[B_SF + wg], kph, abort, a.err, 0x201, (t << 16) | j))) {
         ok = false;
         break;
       }
@@ -299,171 +316,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       float s[64];
       {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_base + S_COL + sb * BN, v);
+        tmem_ld32(tmem + lane_base + S_COL + wg * BN, v);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(v[c]);
-        tmem_ld32(tmem + lane_base + S_COL + sb * BN + 32, v);
+        tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(v[c]);
       }
       tc_fence_before();
-      mbar_arrive(&bar[B_SE + sb]);
+      mbar_arrive(&bar[B_SE + wg]);
+
+      // send this CTA's partial scores into the peer's buffer once the peer's PV of two
+      // blocks ago no longer reads it
+      if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], kph ^ 1, abort, a.err, 0x202,
+                                               (t << 16) | j))) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        st_async_v4(peer_x + q * (TM * 16), __float_as_uint(s[4 * q]),
+                    __float_as_uint(s[4 * q + 1]), __float_as_uint(s[4 * q + 2]),
+                    __float_as_uint(s[4 * q + 3]), peer_xf);
+
       int64_t slot0, g0;
       int valid;
       blk.get(j, slot0, g0, valid);
-
-      if (!owner) {
-        // partial scores of the peer's rows -> peer's exchange buffer
-        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + sb], kph ^ 1, abort, a.err, 0x202,
-                                                 (t << 16) | j))) {
-          ok = false;
-          break;
-        }
-        const uint32_t dst = mapa(smem_u32(sm + OFF_X + sb * X_BYTES), peer) +
-                             (uint32_t)(t - (int)peer * 64) * (BN * 4);
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          st_cluster_v4(dst + q * 16, __float_as_uint(s[4 * q]), __float_as_uint(s[4 * q + 1]),
-                        __float_as_uint(s[4 * q + 2]), __float_as_uint(s[4 * q + 3]));
-        mbar_arrive_cluster(peer_bar(B_XF + sb));
+      if (valid < BN && t < BN && t >= valid) {
         // a partial block: zero this CTA's latent rows past the last key so that masked
-        // keys contribute exact zeros to P.V whatever the ring holds there
-        if (valid < BN) {
-          const int s_idx = j % NST;
-          if (!__all_sync(FULL, mbar_wait(&bar[B_KVF + s_idx], (j / NST) & 1, abort, a.err, 0x203,
-                                          (t << 16) | j))) {
-            ok = false;
-            break;
-          }
-          const int u = t - (int)peer * 64;               // 0..63
-          if (u >= valid) {
-            uint8_t* st = sm + OFF_KV + s_idx * STAGE_BYTES + u * 128;
+        // keys contribute exact zeros to P.V whatever the ring holds there (the stage has
+        // landed: QK of this block has completed)
+        uint8_t* st = sm + OFF_KV + (j % NST) * STAGE_BYTES + t * 128;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4* p = reinterpret_cast<uint4*>(st + q * BOX_BYTES);
+        for (int q = 0; q < 4; ++q) {
+          uint4* p = reinterpret_cast<uint4*>(st + q * BOX_BYTES);
 #pragma unroll
-              for (int w = 0; w < 8; ++w) p[w] = make_uint4(0, 0, 0, 0);
-            }
-          }
+          for (int w = 0; w < 8; ++w) p[w] = make_uint4(0, 0, 0, 0);
         }
-        // this row's P and rescale factor from the owner
-        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_RF + sb], kph, abort, a.err, 0x204,
-                                                 (t << 16) | j))) {
-          ok = false;
-          break;
-        }
-        const float fac = F[sb * TM + t];
-        if (j > 0) {
-          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
-                                          a.err, 0x205, (t << 16) | j))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // warp-collective TMEM access: every lane runs it, factor 1 where nothing grew
-          if (__any_sync(FULL, fac != 1.f)) rescale_row(tmem + lane_base + O_COL, fac);
-          // my P buffer of block j-1 is free again: the peer may write block j+1 rows
-          mbar_arrive_cluster(peer_bar(B_PPE + ((j - 1) & 1)));
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bar[B_PF + sb]);
-      } else {
-        // full scores: add the peer's partial
-        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + sb], kph, abort, a.err, 0x301,
-                                                 (t << 16) | j))) {
-          ok = false;
-          break;
-        }
-        const float4* xr = reinterpret_cast<const float4*>(sm + OFF_X + sb * X_BYTES +
-                                                           (t - (int)rank * 64) * (BN * 4));
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float4 x = xr[q];
-          s[4 * q] += x.x; s[4 * q + 1] += x.y; s[4 * q + 2] += x.z; s[4 * q + 3] += x.w;
-        }
-        mbar_arrive_cluster(peer_bar(B_XE + sb));
-        float mb = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool vis = c < valid && g0 + c < k_end_row;
-          s[c] = vis ? s[c] * a.scale_log2 : -INFINITY;
-          mb = fmaxf(mb, s[c]);
-        }
-        float fac = 1.f;
-        if (j == 0) {
-          m = mb;
-        } else if (mb > m + 8.f) {
-          fac = exp2f(m - mb);
-          m = mb;
-        }
-        const float msub = m == -INFINITY ? 0.f : m;
-        uint32_t pk[32];
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = exp2f(s[2 * c] - msub), p1 = exp2f(s[2 * c + 1] - msub);
-          sum += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
-        }
-        l = l * fac + sum;
-        // warp-collective TMEM access: the whole warp rescales if any of its rows grew
-        if (j > 0 && __any_sync(FULL, fac != 1.f)) {
-          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
-                                          a.err, 0x302, (t << 16) | j))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          rescale_row(tmem + lane_base + O_COL, fac);
-        } else if (j >= 2) {
-          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + sb], kph ^ 1, abort, a.err, 0x303,
-                                          (t << 16) | j))) {
-            ok = false;
-            break;
-          }
-        }
-        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_PPE + sb], kph ^ 1, abort, a.err, 0x304,
-                                                 (t << 16) | j))) {
-          ok = false;
-          break;
-        }
-        uint8_t* prow = sm + OFF_P + sb * P_BYTES + t * 128;
-        const uint32_t prem = mapa(smem_u32(prow), peer);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int pos = (c ^ (t & 7)) * 16;
-          *reinterpret_cast<uint4*>(prow + pos) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          st_cluster_v4(prem + pos, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        st_cluster_f32(mapa(smem_u32(&F[sb * TM + t]), peer), fac);
-        fence_proxy_async_cluster();
-        fence_proxy_async_smem();
-        mbar_arrive_cluster(peer_bar(B_RF + sb));
-        tc_fence_before();
-        mbar_arrive(&bar[B_PF + sb]);
       }
+
+      // full scores: add the peer's partial
+      if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + wg], kph, abort, a.err, 0x203,
+                                               (t << 16) | j))) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 x = my_x[q * TM];
+        s[4 * q] += x.x; s[4 * q + 1] += x.y; s[4 * q + 2] += x.z; s[4 * q + 3] += x.w;
+      }
+      named_bar(1 + wg, TM);            // the whole buffer is read before P overwrites it
+
+      // masked raw maximum (scores are scaled inside the exponent)
+      const int64_t lim64 = k_end_row - g0;
+      const int lim = lim64 < valid ? (lim64 < 0 ? 0 : (int)lim64) : valid;
+      if (lim < BN) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+      }
+      float rmax = s[0];
+#pragma unroll
+      for (int c = 1; c < 64; ++c) rmax = fmaxf(rmax, s[c]);
+      const float mb = rmax * c2;
+
+      // running maximum after the previous block (published by the other warpgroup)
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        if (!__all_sync(FULL, mbar_wait(&bar[B_M + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
+                                        a.err, 0x204, (t << 16) | j))) {
+          ok = false;
+          break;
+        }
+        m_prev = m_sh[((j - 1) & 1) * TM + t];
+      }
+      float m = m_prev, fac = 1.f;
+      if (j == 0) {
+        m = mb;
+      } else if (mb > m_prev + 8.f) {
+        m = mb;
+        fac = ex2(m_prev - m);
+      }
+      m_sh[wg * TM + t] = m;
+      mbar_arrive(&bar[B_M + wg]);
+
+      const float msub = m == -INFINITY ? 0.f : m;
+      uint32_t pk[32];
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2(fmaf(s[2 * c], c2, -msub));
+        const float p1 = ex2(fmaf(s[2 * c + 1], c2, -msub));
+        sum += p0 + p1;
+        pk[c] = pack_bf16(p0, p1);
+      }
+      l = l * ex2(m_last - msub) + sum;
+      m_last = m;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+
+      // warp-collective TMEM access: the whole warp rescales O if any of its rows grew
+      if (j > 0 && __any_sync(FULL, fac != 1.f)) {
+        if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
+                                        a.err, 0x205, (t << 16) | j))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        rescale_row(tmem + lane_base + O_COL, fac);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar[B_PF + wg]);
     }
 
     // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait(&bar[B_DONE], 0, abort, a.err, 0x401, t);
+    ok = __all_sync(FULL, ok);
     tc_fence_after();
-    float inv = 0.f;
-    if (owner) {
-      inv = l > 0.f ? 1.f / l : 0.f;
-      st_cluster_f32(mapa(smem_u32(&F[2 * TM + t]), peer), inv);
-      mbar_arrive_cluster(peer_bar(B_FIN));
-      if (a.lse && row_valid && ok) a.lse[grow] = (m + log2f(l)) * 0.69314718055994530942f;
-    } else {
-      if (ok) ok = mbar_wait_cluster(&bar[B_FIN], 0, abort, a.err, 0x402, t);
-      inv = F[2 * TM + t];
-    }
+    l_sh[(wg * 2) * TM + t] = l;
+    l_sh[(wg * 2 + 1) * TM + t] = m_last;
+    named_bar(3, 2 * TM);
+    const float l0 = l_sh[t], m0 = l_sh[TM + t], l1 = l_sh[2 * TM + t], m1 = l_sh[3 * TM + t];
+    const float mf = fmaxf(m0, m1);
+    const float lt = l0 * ex2(m0 - mf) + l1 * ex2(m1 - mf);
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    if (wg == 0 && rank == 0 && a.lse && row_valid && ok)
+      a.lse[grow] = (mf + log2f(lt)) * 0.69314718055994530942f;
     bf16* dst = a.o_lat + grow * G.Dc + rank * HALF;
 #pragma unroll 1
-    for (int c = 0; c < HALF; c += 32) {
+    for (int c = wg * (HALF / 2); c < (wg + 1) * (HALF / 2); c += 32) {
       uint32_t v[32];
       tmem_ld32(tmem + lane_base + O_COL + c, v);
       tmem_wait_ld();
@@ -487,7 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   __syncthreads();
   __syncwarp();
   cluster_sync();          // no remote access into this CTA is still pending
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -530,7 +516,7 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
   a.err = err;
   const int64_t tiles = (int64_t)g.B * a.tiles_per_batch;
-  attend_kernel<<<(unsigned)(2 * tiles), 192, ATT_SMEM, st>>>(K, Q, a);
+  attend_kernel<<<(unsigned)(2 * tiles), NTHREADS, ATT_SMEM, st>>>(K, Q, a);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;

@@ -11,10 +11,10 @@
 //   - TMA-loads its columns of the 64 cached rows (one load serves as K and as V),
 //   - computes its partial score S_c = Q_c . K_c^T with tcgen05.mma (Q's latent half
 //     resident in TMEM as the A operand, the RoPE part from shared memory),
-//   - swaps partial scores with its peer through distributed shared memory, so both
-//     CTAs hold the full scores of all 128 rows,
+//   - swaps partial scores (rounded to fp16) with its peer through distributed shared
+//     memory, so both CTAs hold the full scores of all 128 rows,
 //   - runs the online softmax of all 128 rows itself (both CTAs take bit-identical
-//     decisions: the same fp32 sums in the same order),
+//     decisions: each adds the same two fp16-rounded partials),
 //   - accumulates O_c += P . V_c (M=128, N=256) into its TMEM.
 //
 // Two softmax warpgroups take alternate key blocks, so the exchange of one block
@@ -32,6 +32,8 @@
 #include "tc_ptx.cuh"
 #include "tmap.h"
 
+#include <cuda_fp16.h>
+
 namespace mla {
 namespace {
 
@@ -39,15 +41,15 @@ using namespace tc;
 
 constexpr int TM = 128;                               // rows per tile
 constexpr int BN = 64;                                // keys per block
-constexpr int NST = 3;                                // K/V pipeline stages
+constexpr int NST = 4;                                // K/V pipeline stages
 constexpr int HALF = 256;                             // latent dims per CTA
 constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
 constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB
 constexpr int STAGE_BYTES = LAT_BYTES + BOX_BYTES;    // + RoPE box (CTA 1)
 constexpr int QR_BYTES = TM * 64 * 2;                 // Q RoPE part, 16 KB
-constexpr int X_BYTES = TM * BN * 4;                  // exchange buffer, 32 KB: the peer's
-                                                      // partial scores, chunk-major
-                                                      // [16 x float4][128 rows]; then P
+constexpr int X_BYTES = TM * BN * 2;                  // exchange buffer, 16 KB: the peer's
+                                                      // partial scores as fp16, chunk-major
+                                                      // [8 x 16 B][128 rows]; then P
                                                       // (bf16, 128-byte swizzled rows)
 constexpr int NTHREADS = 320;
 
@@ -298,7 +300,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
     const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * X_BYTES), peer) + (uint32_t)t * 16;
     const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
-    const float4* my_x = reinterpret_cast<const float4*>(sm + OFF_X + wg * X_BYTES) + t;
+    const uint4* my_x = reinterpret_cast<const uint4*>(sm + OFF_X + wg * X_BYTES) + t;
     uint8_t* prow = sm + OFF_X + wg * X_BYTES + t * 128;     // P row t over the same buffer
     const float c2 = a.scale_log2;
     float m_last = -INFINITY, l = 0.f;         // this warpgroup's running sum and its max
@@ -335,11 +337,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         ok = false;
         break;
       }
+      // both CTAs add the same two fp16-rounded partials, so their softmax agrees bit
+      // for bit; the rounding is ~2^-11 of a partial score
+      uint32_t hs[32];
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        st_async_v4(peer_x + q * (TM * 16), __float_as_uint(s[4 * q]),
-                    __float_as_uint(s[4 * q + 1]), __float_as_uint(s[4 * q + 2]),
-                    __float_as_uint(s[4 * q + 3]), peer_xf);
+      for (int c = 0; c < 32; ++c) {
+        __half2 h2 = __floats2half2_rn(s[2 * c], s[2 * c + 1]);
+        hs[c] = *reinterpret_cast<uint32_t*>(&h2);
+        const float2 back = __half22float2(h2);
+        s[2 * c] = back.x;
+        s[2 * c + 1] = back.y;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st_async_v4(peer_x + q * (TM * 16), hs[4 * q], hs[4 * q + 1], hs[4 * q + 2],
+                    hs[4 * q + 3], peer_xf);
 
       int64_t slot0, g0;
       int valid;
@@ -364,9 +376,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         break;
       }
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float4 x = my_x[q * TM];
-        s[4 * q] += x.x; s[4 * q + 1] += x.y; s[4 * q + 2] += x.z; s[4 * q + 3] += x.w;
+      for (int q = 0; q < 8; ++q) {
+        const uint4 x = my_x[q * TM];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+          s[8 * q + 2 * e] += f.x;
+          s[8 * q + 2 * e + 1] += f.y;
+        }
       }
       named_bar(1 + wg, TM);            // the whole buffer is read before P overwrites it
 

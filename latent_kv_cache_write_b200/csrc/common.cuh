@@ -64,6 +64,43 @@ __device__ __forceinline__ void rope_rotate(float& a, float& b, double ang) {
   b = (float)nb;
 }
 
+// Axis position of token g for RoPE pair p, and the pair's frequency theta^(-j/n).
+__device__ __forceinline__ int64_t rope_pos(const Geo& G, int64_t g, int p) {
+  const int64_t t = g / G.F;
+  const int64_t r = g - t * G.F;
+  if (p < G.pairs[0]) return t;
+  const int64_t y = r / G.gw;
+  if (p < G.pairs[0] + G.pairs[1]) return y;
+  return r - y * G.gw;
+}
+__device__ __forceinline__ double rope_inv_freq(const Geo& G, int p) {
+  int j, n;
+  if (p < G.pairs[0]) {
+    j = p; n = G.pairs[0];
+  } else if (p < G.pairs[0] + G.pairs[1]) {
+    j = p - G.pairs[0]; n = G.pairs[1];
+  } else {
+    j = p - G.pairs[0] - G.pairs[1]; n = G.pairs[2];
+  }
+  return pow(G.theta, -(double)j / (double)n);
+}
+
+// Rotate (a, b) by the angle pos * inv_freq: the product is formed in double, reduced
+// modulo 2*pi in double (Cody-Waite with a two-part 2*pi), then sin/cos are evaluated in
+// single precision; the error is ~1e-7 rad for any position the ABI admits.
+__device__ __forceinline__ void rope_rotate_fast(float& a, float& b, double pos, double inv_freq) {
+  const double ang = pos * inv_freq;
+  const double k = rint(ang * 0.15915494309189535);          // 1 / (2 pi)
+  double r = fma(-k, 6.283185307179586, ang);                 // 2 pi, leading part
+  r = fma(-k, 2.4492935982947064e-16, r);                     // 2 pi, trailing part
+  float s, c;
+  sincosf((float)r, &s, &c);
+  const float na = a * c - b * s;
+  const float nb = a * s + b * c;
+  a = na;
+  b = nb;
+}
+
 __device__ __forceinline__ void set_device_error(unsigned int* err, unsigned int code) {
   if (err) atomicOr(err, code);
 }

@@ -44,8 +44,12 @@ constexpr int BN = 64;                                // keys per block
 constexpr int NST = 4;                                // K/V pipeline stages
 constexpr int HALF = 256;                             // latent dims per CTA
 constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
-constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB
+constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB of latent per stage
 constexpr int STAGE_BYTES = LAT_BYTES + BOX_BYTES;    // + RoPE box (CTA 1)
+// Shared-memory K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half)
+// of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage s at OFF_KVR +
+// s * BOX_BYTES.  Stages 2i and 2i+1 are adjacent within every box column, so one
+// N=128 score MMA covers two consecutive 64-key blocks.
 constexpr int QR_BYTES = TM * 64 * 2;                 // Q RoPE part, 16 KB
 constexpr int X_BYTES = TM * BN * 2;                  // exchange buffer, 16 KB: the peer's
                                                       // partial scores as fp16, chunk-major
@@ -54,6 +58,7 @@ constexpr int X_BYTES = TM * BN * 2;                  // exchange buffer, 16 KB:
 constexpr int NTHREADS = 320;
 
 constexpr int OFF_KV = 0;
+constexpr int OFF_KVR = OFF_KV + NST * LAT_BYTES;
 constexpr int OFF_QR = OFF_KV + NST * STAGE_BYTES;
 constexpr int OFF_X = OFF_QR + QR_BYTES;              // [2] exchange / P buffers
 constexpr int OFF_M = OFF_X + 2 * X_BYTES;            // running max handoff [2][128]
@@ -206,64 +211,115 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         int64_t slot0, g0;
         int valid;
         blk.get(j, slot0, g0, valid);
-        uint8_t* st = sm + OFF_KV + s * STAGE_BYTES;
         mbar_expect_tx(&bar[B_KVF + s], bytes);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          tma_load_3d(st + q * BOX_BYTES, &tmK, &bar[B_KVF + s], (int)rank * HALF + q * 64,
-                      (int32_t)slot0, b);
+          tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
+                      (int)rank * HALF + q * 64, (int32_t)slot0, b);
         if (rank == 1)
-          tma_load_3d(st + LAT_BYTES, &tmK, &bar[B_KVF + s], G.Dc, (int32_t)slot0, b);
+          tma_load_3d(sm + OFF_KVR + s * BOX_BYTES, &tmK, &bar[B_KVF + s], G.Dc,
+                      (int32_t)slot0, b);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Scores of blocks 2i and 2i+1 are one N=128 series (S buffers 0 and 1 are adjacent);
+    // a score series is issued as soon as its data and S buffers are ready, since the
+    // scores start the softmax chains.  PV products are issued in block order, as soon as
+    // their P is ready whenever the issuer would otherwise wait: that frees the K/V stage
+    // for the next load and the exchange buffer for the peer early.
     if (lane == 0) {
-      const uint32_t id_qk = idesc_bf16(128, BN, false, false);
+      const uint32_t id_qk = idesc_bf16(128, 2 * BN, false, false);
       const uint32_t id_pv = idesc_bf16(128, HALF, false, true);
       bool ok = mbar_wait(&bar[B_QREADY], 0, abort, a.err, 0x102, 0);
       if (ok && rank == 1) ok = mbar_wait(&bar[B_QR], 0, abort, a.err, 0x103, 0);
       tc_fence_after();
-      auto pv = [&](int jj) -> bool {
+      int next_pv = 0;                         // next block whose PV is to be issued
+      auto issue_pv = [&](int jj) {
         const int pb = jj & 1;
-        if (!mbar_wait(&bar[B_PF + pb], (jj >> 1) & 1, abort, a.err, 0x104, jj)) return false;
+        const int s = jj % NST;
         tc_fence_after();
-        const uint32_t st = smem_u32(sm + OFF_KV + (jj % NST) * STAGE_BYTES);
+        const uint32_t v0 = smem_u32(sm + OFF_KV + s * BOX_BYTES);
         const uint32_t pa = smem_u32(sm + OFF_X + pb * X_BYTES);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
-                 desc_sw128(st + ks * 2048, BOX_BYTES, 1024), id_pv, (jj > 0 || ks > 0) ? 1u : 0u);
+                 desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
+                 (jj > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bar[B_PE + pb]);
-        mma_commit(&bar[B_KVE + jj % NST]);
+        mma_commit(&bar[B_KVE + s]);
         // the peer's warpgroup waits for this before refilling the buffer at block jj+2;
         // no signal is sent that nobody waits for (the peer may have exited by then)
         if (jj + 2 < nblk) mma_commit_cluster(&bar[B_XE + pb], (uint16_t)(1u << peer));
-        return true;
       };
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int s = j % NST, sb = j & 1;
-        if (!mbar_wait(&bar[B_KVF + s], (j / NST) & 1, abort, a.err, 0x105, j)) break;
-        if (!mbar_wait(&bar[B_SE + sb], ((j >> 1) & 1) ^ 1, abort, a.err, 0x106, j)) break;
+      // issue every PV whose P is ready, for blocks below `limit`, without blocking
+      auto pv_ready = [&](int limit) {
+        while (next_pv < limit &&
+               mbar_test_wait(&bar[B_PF + (next_pv & 1)], (next_pv >> 1) & 1)) {
+          issue_pv(next_pv);
+          ++next_pv;
+        }
+      };
+      // wait for a phase while keeping the PV stream moving
+      auto wait_pv = [&](uint64_t* w, uint32_t parity, int limit, uint32_t site, int j) -> bool {
+        if (mbar_test_wait(w, parity)) return true;
+        const long long c0 = clock64();
+        for (uint32_t it = 1;; ++it) {
+          pv_ready(limit);
+          if (mbar_test_wait(w, parity)) return true;
+          if ((it & 255u) == 0) {
+            if (*abort) return false;
+            if (clock64() - c0 > 4000000000ll) {
+              *abort = 1;
+              report_timeout(a.err, site, (uint32_t)j);
+              return false;
+            }
+          }
+        }
+      };
+      const int npair = (nblk + 1) / 2;
+      for (int i = 0; ok && i < npair; ++i) {
+        const int j0 = 2 * i, s0 = j0 % NST;
+        const bool two = j0 + 1 < nblk;
+        const uint32_t ph = (i & 1) ^ 1;
+        if (!wait_pv(&bar[B_KVF + s0], (j0 / NST) & 1, j0, 0x105, j0)) { ok = false; break; }
+        if (two && !wait_pv(&bar[B_KVF + s0 + 1], (j0 / NST) & 1, j0, 0x105, j0 + 1)) {
+          ok = false;
+          break;
+        }
+        if (!wait_pv(&bar[B_SE], ph, j0, 0x106, j0)) { ok = false; break; }
+        if (!wait_pv(&bar[B_SE + 1], ph, j0, 0x106, j0 + 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d = tmem + S_COL + sb * BN;
-        const uint32_t st = smem_u32(sm + OFF_KV + s * STAGE_BYTES);
+        const uint32_t d = tmem + S_COL;
+        const uint32_t k0 = smem_u32(sm + OFF_KV + s0 * BOX_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < HALF / 16; ++kk)
+        for (int kk = 0; kk < HALF / 16; ++kk) {
           mma_ts(d, tmem + Q_COL + kk * 8,
-                 desc_sw128(st + (kk >> 2) * BOX_BYTES + (kk & 3) * 32, 16, 1024), id_qk,
+                 desc_sw128(k0 + (kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32, 16, 1024), id_qk,
                  kk > 0 ? 1u : 0u);
+        }
         if (rank == 1) {
           const uint32_t qa = smem_u32(sm + OFF_QR);
+          const uint32_t kr = smem_u32(sm + OFF_KVR + s0 * BOX_BYTES);
 #pragma unroll
           for (int w = 0; w < 4; ++w)
-            mma_ss(d, desc_sw128(qa + w * 32, 16, 1024),
-                   desc_sw128(st + LAT_BYTES + w * 32, 16, 1024), id_qk, 1u);
+            mma_ss(d, desc_sw128(qa + w * 32, 16, 1024), desc_sw128(kr + w * 32, 16, 1024),
+                   id_qk, 1u);
         }
-        mma_commit(&bar[B_SF + sb]);
-        if (j > 0 && !pv(j - 1)) { ok = false; break; }
+        mma_commit(&bar[B_SF]);
+        mma_commit(&bar[B_SF + 1]);
+        pv_ready(j0);
       }
-      if (ok && nblk > 0) pv(nblk - 1);
+      // remaining PV products
+      while (ok && next_pv < nblk) {
+        if (!mbar_wait(&bar[B_PF + (next_pv & 1)], (next_pv >> 1) & 1, abort, a.err, 0x104,
+                       next_pv)) {
+          ok = false;
+          break;
+        }
+        issue_pv(next_pv);
+        ++next_pv;
+      }
       mma_commit(&bar[B_DONE]);
     }
   } else {
@@ -360,10 +416,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // a partial block: zero this CTA's latent rows past the last key so that masked
         // keys contribute exact zeros to P.V whatever the ring holds there (the stage has
         // landed: QK of this block has completed)
-        uint8_t* st = sm + OFF_KV + (j % NST) * STAGE_BYTES + t * 128;
+        uint8_t* st = sm + OFF_KV + (j % NST) * BOX_BYTES + t * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint4* p = reinterpret_cast<uint4*>(st + q * BOX_BYTES);
+          uint4* p = reinterpret_cast<uint4*>(st + q * NST * BOX_BYTES);
 #pragma unroll
           for (int w = 0; w < 8; ++w) p[w] = make_uint4(0, 0, 0, 0);
         }

@@ -2,10 +2,12 @@
 //   cache write:  [h] x [W_DKV | W_KR]  -> RoPE on the W_KR columns -> bf16 -> ring slot
 //   absorb:       q_nope[:, h] x W_UK[h] -> q_lat (plus RoPE of q_R in the same CTAs)
 //   up-projection: o_lat[:, h] x W_UV[h]^T -> out
-// One 128 x BN output tile per CTA.  Warp 0 lane 0 issues TMA loads into a 4-stage
-// shared-memory ring, warp 1 lane 0 issues tcgen05.mma (M=128, N=BN, K=16 steps) into a
-// TMEM accumulator; afterwards all four warps read the accumulator (one row per
-// thread) and run the fused epilogue.
+// Persistent: one CTA per SM walks the 128 x 128 output tiles (M fastest, so CTAs that
+// run together share the weight tile in L2).  Warp 0 lane 0 streams TMA loads through a
+// 4-stage shared-memory ring, warp 1 lane 0 issues tcgen05.mma (M=128, N=128, K=16 steps)
+// into one of two TMEM accumulators, and warps 2-5 drain the other accumulator (one row
+// per thread) through the fused epilogue, so a tile's epilogue overlaps the next tile's
+// main loop.
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tmap.h"
@@ -16,15 +18,17 @@ namespace {
 using namespace tc;
 
 constexpr int GBM = 128, GBK = 64, GSTAGES = 4, GBN = 128;
+constexpr int GTHREADS = 192;
 constexpr int A_BYTES = GBM * GBK * 2;           // 16 KB
 constexpr int B_BYTES = GBN * GBK * 2;           // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GEMM_SMEM = GSTAGES * STAGE_BYTES + 1024 + 256;
+constexpr int MAX_PAIRS = 512;                   // RoPE pairs with a table entry (d_R <= 1024)
+constexpr int GEMM_SMEM = GSTAGES * STAGE_BYTES + 1024 + 256 + MAX_PAIRS * 8;
 
 enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
 
 struct TcGemm {
-  int M, N, K;
+  int M, N, K, Z;
   int mode;
   int b_mn;                 // B is MN-major (N contiguous) instead of K-major
   int n_split;              // cache: tiles at n >= n_split read tmB2 at n - n_split
@@ -37,7 +41,7 @@ struct TcGemm {
   unsigned int* err;
 };
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(GTHREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, TcGemm p) {
   extern __shared__ uint8_t smem_raw[];
@@ -45,152 +49,210 @@ __global__ void __launch_bounds__(128, 1)
                                              ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + GSTAGES * STAGE_BYTES);
   uint64_t* empty = full + GSTAGES;
-  uint64_t* done = empty + GSTAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* accf = empty + GSTAGES;              // accumulator ready [2]
+  uint64_t* acce = accf + 2;                     // accumulator drained [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  double* inv_freq = reinterpret_cast<double*>(smem + GSTAGES * STAGE_BYTES + 256);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * GBM, n0 = blockIdx.y * GBN, z = blockIdx.z;
-  const bool second = p.mode == MODE_CACHE && n0 >= p.n_split;
-  const CUtensorMap* mB = second ? &tmB2 : &tmB;
-  const int nb = second ? n0 - p.n_split : n0;
+  const int nm = (p.M + GBM - 1) / GBM, nn = (p.N + GBN - 1) / GBN;
+  const int ntiles = nm * nn * p.Z;
+  const int nk = (p.K + GBK - 1) / GBK;
 
   if (tid == 0) {
     for (int s = 0; s < GSTAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 128);
+    }
     *abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
-    prefetch_tmap(mB);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmB2);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, GBN);
+    tmem_alloc(tmem_slot, 2 * GBN);
     tmem_relinquish();
   }
+  for (int q = tid; q < p.geo.Dr / 2 && q < MAX_PAIRS; q += GTHREADS)
+    inv_freq[q] = rope_inv_freq(p.geo, q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nk = (p.K + GBK - 1) / GBK;
 
-  if (warp == 0 && lane == 0) {
-    // TMA producer
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % GSTAGES;
-      const uint32_t ph = (kb / GSTAGES) & 1;
-      if (!mbar_wait(&empty[s], ph ^ 1, abort, p.err, 0x11, kb)) break;
-      uint8_t* a = smem + s * STAGE_BYTES;
-      uint8_t* b = a + A_BYTES;
-      mbar_expect_tx(&full[s], STAGE_BYTES);
-      tma_load_3d(a, &tmA, &full[s], kb * GBK, p.mode == MODE_CACHE ? 0 : z, m0);
-      if (p.b_mn) {
-        tma_load_3d(b, mB, &full[s], nb, kb * GBK, z);
-        tma_load_3d(b + B_BYTES / 2, mB, &full[s], nb + 64, kb * GBK, z);
-      } else {
-        tma_load_3d(b, mB, &full[s], kb * GBK, nb, z);
+  auto tile_coords = [&](int t, int& m0, int& n0, int& z) {
+    z = t / (nm * nn);
+    const int r = t - z * nm * nn;
+    m0 = (r % nm) * GBM;
+    n0 = (r / nm) * GBN;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        int m0, n0, z;
+        tile_coords(t, m0, n0, z);
+        const bool second = p.mode == MODE_CACHE && n0 >= p.n_split;
+        const CUtensorMap* mB = second ? &tmB2 : &tmB;
+        const int nb = second ? n0 - p.n_split : n0;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % GSTAGES;
+          if (!mbar_wait(&empty[s], ((it / GSTAGES) & 1) ^ 1, abort, p.err, 0x11, kb)) break;
+          uint8_t* a = smem + s * STAGE_BYTES;
+          uint8_t* b = a + A_BYTES;
+          mbar_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_3d(a, &tmA, &full[s], kb * GBK, p.mode == MODE_CACHE ? 0 : z, m0);
+          if (p.b_mn) {
+            tma_load_3d(b, mB, &full[s], nb, kb * GBK, z);
+            tma_load_3d(b + B_BYTES / 2, mB, &full[s], nb + 64, kb * GBK, z);
+          } else {
+            tma_load_3d(b, mB, &full[s], kb * GBK, nb, z);
+          }
+        }
+        if (*abort) break;
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer
-    const uint32_t idesc = idesc_bf16(GBM, GBN, false, p.b_mn != 0);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % GSTAGES;
-      const uint32_t ph = (kb / GSTAGES) & 1;
-      if (!mbar_wait(&full[s], ph, abort, p.err, 0x12, kb)) break;
-      tc_fence_after();
-      const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
-      const uint32_t b = a + A_BYTES;
-      const uint64_t da = desc_sw128(a, 16, 1024);
-      const uint64_t db = p.b_mn ? desc_sw128(b, B_BYTES / 2, 1024) : desc_sw128(b, 16, 1024);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(GBM, GBN, false, p.b_mn != 0);
+      uint32_t it = 0, tc = 0;
+      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+        const int acc = tc & 1;
+        if (!mbar_wait(&acce[acc], ((tc >> 1) & 1) ^ 1, abort, p.err, 0x14, tc)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * GBN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % GSTAGES;
+          if (!mbar_wait(&full[s], (it / GSTAGES) & 1, abort, p.err, 0x12, kb)) break;
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b = a + A_BYTES;
+          const uint64_t da = desc_sw128(a, 16, 1024);
+          const uint64_t db = p.b_mn ? desc_sw128(b, B_BYTES / 2, 1024) : desc_sw128(b, 16, 1024);
 #pragma unroll
-      for (int ks = 0; ks < GBK / 16; ++ks) {
-        // K-major operands advance 32 bytes per 16-element K step inside the swizzle
-        // atom; the MN-major B advances 16 rows of 128 bytes.
-        const uint64_t bstep = p.b_mn ? (uint64_t)(ks * 2048 >> 4) : (uint64_t)(ks * 32 >> 4);
-        mma_ss(tmem, da + (uint64_t)(ks * 32 >> 4), db + bstep, idesc, (kb | ks) != 0);
+          for (int ks = 0; ks < GBK / 16; ++ks) {
+            // K-major operands advance 32 bytes per 16-element K step inside the swizzle
+            // atom; the MN-major B advances 16 rows of 128 bytes.
+            const uint64_t bstep = p.b_mn ? (uint64_t)(ks * 2048 >> 4) : (uint64_t)(ks * 32 >> 4);
+            mma_ss(d, da + (uint64_t)(ks * 32 >> 4), db + bstep, idesc, (kb | ks) != 0);
+          }
+          mma_commit(&empty[s]);
+        }
+        mma_commit(&accf[acc]);
+        if (*abort) break;
       }
-      mma_commit(&empty[s]);
     }
-    mma_commit(done);
+  } else {
+    // ---------------------------------------------------------------- epilogue warps
+    const int r = (warp & 3) * 32 + lane;       // TMEM lane quarter = warp id % 4
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const Geo& G = p.geo;
+    uint32_t tc = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+      int m0, n0, z;
+      tile_coords(t, m0, n0, z);
+      const int acc = tc & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[acc], (tc >> 1) & 1, abort, p.err,
+                                                         0x13, (r << 16) | tc));
+      tc_fence_after();
+      const int64_t m = m0 + r;
+      const uint32_t trow = tmem + lane_base + acc * GBN;
+      for (int c0 = 0; c0 < GBN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c0, v);
+        tmem_wait_ld();
+        if (c0 + 32 == GBN) {
+          tc_fence_before();
+          mbar_arrive(&acce[acc]);              // accumulator may be overwritten
+        }
+        if (!ok || m >= p.M) continue;
+        const int n = n0 + c0;                  // output column of v[0]
+        if (n >= p.N) continue;
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+        bf16* dst;
+        if (p.mode == MODE_CACHE) {
+          const int64_t b = m / p.rows_per_batch;
+          const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
+          const int64_t slot = g % G.S;
+          if (n >= p.n_split) {
+#pragma unroll 4
+            for (int j = 0; j < 32; j += 2) {
+              const int q = (n + j - p.n_split) / 2;
+              rope_rotate_fast(f[j], f[j + 1], (double)rope_pos(G, g, q), inv_freq[q]);
+            }
+          }
+          dst = p.out + (b * G.S + slot) * G.row + n;
+        } else if (p.mode == MODE_ABSORB) {
+          dst = p.out + (m * G.H + z) * G.row + n;
+        } else {
+          dst = p.out + (m * G.H + z) * G.Dn + n;
+        }
+        const int valid = p.N - n < 32 ? p.N - n : 32;
+        if (valid == 32) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16(f[8 * q + 0], f[8 * q + 1]);
+            w.y = pack_bf16(f[8 * q + 2], f[8 * q + 3]);
+            w.z = pack_bf16(f[8 * q + 4], f[8 * q + 5]);
+            w.w = pack_bf16(f[8 * q + 6], f[8 * q + 7]);
+            reinterpret_cast<uint4*>(dst)[q] = w;
+          }
+        } else {
+          for (int j = 0; j < valid; ++j) dst[j] = __float2bfloat16_rn(f[j]);
+        }
+      }
+      if (ok && m < p.M && n0 == 0) {
+        if (p.mode == MODE_CACHE && p.slots) {
+          const int64_t b = m / p.rows_per_batch;
+          const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
+          p.slots[m] = (int32_t)(g % G.S);
+        }
+        if (p.mode == MODE_ABSORB && G.Dr > 0) {
+          // q_abs[.., Dc:] = RoPE(q_R) for this tile's rows and head
+          const int64_t i = m % p.rows_per_batch;
+          const int64_t g = p.first_tok + i;
+          const bf16* src = p.q_rope + (m * G.H + z) * G.Dr;
+          bf16* dst = p.out + (m * G.H + z) * G.row + G.Dc;
+          for (int q = 0; q < G.Dr / 2; ++q) {
+            float a = __bfloat162float(src[2 * q]), b = __bfloat162float(src[2 * q + 1]);
+            rope_rotate_fast(a, b, (double)rope_pos(G, g, q), inv_freq[q]);
+            *reinterpret_cast<uint32_t*>(dst + 2 * q) = pack_bf16(a, b);
+          }
+        }
+      }
+      if (!ok) break;
+    }
   }
   __syncwarp();
-
-  // ---------------------------------------------------------------- epilogue
-  const bool ok = mbar_wait(done, 0, abort, p.err, 0x13, tid);
-  tc_fence_after();
-  const int r = warp * 32 + lane;
-  const int64_t m = m0 + r;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-  const Geo& G = p.geo;
-  for (int c0 = 0; c0 < GBN; c0 += 32) {
-    uint32_t v[32];
-    tmem_ld32(trow + c0, v);
-    tmem_wait_ld();
-    if (!ok || m >= p.M) continue;
-    const int n = n0 + c0;                        // output column of v[0]
-    if (n >= p.N) continue;
-    float f[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-    bf16* dst;
-    if (p.mode == MODE_CACHE) {
-      const int64_t b = m / p.rows_per_batch;
-      const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
-      const int64_t slot = g % G.S;
-      if (n >= p.n_split) {
-#pragma unroll 4
-        for (int j = 0; j < 32; j += 2)
-          rope_rotate(f[j], f[j + 1], rope_angle(G, g, (n + j - p.n_split) / 2));
-      }
-      dst = p.out + (b * G.S + slot) * G.row + n;
-    } else if (p.mode == MODE_ABSORB) {
-      dst = p.out + (m * G.H + z) * G.row + n;
-    } else {
-      dst = p.out + (m * G.H + z) * G.Dn + n;
-    }
-    const int valid = p.N - n < 32 ? p.N - n : 32;
-    if (valid == 32) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        w.x = pack_bf16(f[8 * q + 0], f[8 * q + 1]);
-        w.y = pack_bf16(f[8 * q + 2], f[8 * q + 3]);
-        w.z = pack_bf16(f[8 * q + 4], f[8 * q + 5]);
-        w.w = pack_bf16(f[8 * q + 6], f[8 * q + 7]);
-        reinterpret_cast<uint4*>(dst)[q] = w;
-      }
-    } else {
-      for (int j = 0; j < valid; ++j) dst[j] = __float2bfloat16_rn(f[j]);
-    }
-  }
-  if (ok && m < p.M && blockIdx.y == 0) {
-    if (p.mode == MODE_CACHE && p.slots) {
-      const int64_t b = m / p.rows_per_batch;
-      const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
-      p.slots[m] = (int32_t)(g % G.S);
-    }
-    if (p.mode == MODE_ABSORB && G.Dr > 0) {
-      // q_abs[.., Dc:] = RoPE(q_R) for this CTA's rows and head
-      const int64_t i = m % p.rows_per_batch;
-      const int64_t g = p.first_tok + i;
-      const bf16* src = p.q_rope + (m * G.H + z) * G.Dr;
-      bf16* dst = p.out + (m * G.H + z) * G.row + G.Dc;
-      for (int q = 0; q < G.Dr / 2; ++q) {
-        float a = __bfloat162float(src[2 * q]), b = __bfloat162float(src[2 * q + 1]);
-        rope_rotate(a, b, rope_angle(G, g, q));
-        *reinterpret_cast<uint32_t*>(dst + 2 * q) = pack_bf16(a, b);
-      }
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, GBN);
+    tmem_dealloc(tmem, 2 * GBN);
   }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
 }
 
 cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
@@ -202,8 +264,13 @@ cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid((p.M + GBM - 1) / GBM, (p.N + GBN - 1) / GBN, zcount);
-  tc_gemm_kernel<<<grid, 128, GEMM_SMEM, st>>>(A, B, B2, p);
+  TcGemm q = p;
+  q.Z = zcount;
+  const long long tiles =
+      (long long)((p.M + GBM - 1) / GBM) * ((p.N + GBN - 1) / GBN) * zcount;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (grid == 0) return cudaSuccess;
+  tc_gemm_kernel<<<grid, GTHREADS, GEMM_SMEM, st>>>(A, B, B2, q);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;
@@ -212,7 +279,7 @@ cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap
 }  // namespace
 
 bool tc_gemm_supported(const Geo& g, int d_model) {
-  return g.Dc % GBN == 0 && g.Dr % 64 == 0 && g.Dn % 64 == 0 &&
+  return g.Dc % GBN == 0 && g.Dr % 64 == 0 && g.Dn % 64 == 0 && g.Dr / 2 <= MAX_PAIRS &&
          (d_model <= 0 || d_model % 64 == 0);
 }
 

@@ -5,9 +5,9 @@
 // dims): S = Q_abs . [c || k_R]^T, P = softmax(S), O_lat = P . c.
 //
 // A 128 x 512 fp32 output accumulator fills a whole SM's tensor memory, so each 128-row
-// tile is handled by a cluster of two CTAs that split the latent dimension: CTA 0 owns
-// latent dims [0, 256), CTA 1 owns [256, 512) plus the 64 RoPE dims.  Per block of 64
-// keys each CTA
+// tile is handled by a cluster of two CTAs that split the latent dimension: CTA c owns
+// latent dims [256c, 256c + 256) and RoPE dims [32c, 32c + 32).  Per block of 64 keys
+// each CTA
 //   - TMA-loads its columns of the 64 cached rows (one load serves as K and as V),
 //   - computes its partial score S_c = Q_c . K_c^T with tcgen05.mma (Q's latent half
 //     resident in TMEM as the A operand, the RoPE part from shared memory),
@@ -19,10 +19,8 @@
 //
 // Two softmax warpgroups take alternate key blocks, so the exchange of one block
 // overlaps the exponentials of the other; they hand the running row maximum to each
-// other through shared memory.  P (bf16) is written over the block's consumed exchange
-// buffer; the peer may refill that buffer once the PV product reading it has finished,
-// which the MMA thread signals straight into the peer's barrier with a multicast
-// tcgen05.commit.  O is rescaled only when a row maximum grows by more than 8 (log2
+// other through shared memory.  An exchange buffer is handed back to the peer as soon as
+// its scores are read.  O is rescaled only when a row maximum grows by more than 8 (log2
 // units).  Masking is frame-block-causal per row; a ring that wraps is walked as two
 // contiguous slot segments.
 //
@@ -45,23 +43,25 @@ constexpr int NST = 4;                                // K/V pipeline stages
 constexpr int HALF = 256;                             // latent dims per CTA
 constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
 constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB of latent per stage
-constexpr int STAGE_BYTES = LAT_BYTES + BOX_BYTES;    // + RoPE box (CTA 1)
-// Shared-memory K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half)
-// of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage s at OFF_KVR +
-// s * BOX_BYTES.  Stages 2i and 2i+1 are adjacent within every box column, so one
-// N=128 score MMA covers two consecutive 64-key blocks.
-constexpr int QR_BYTES = TM * 64 * 2;                 // Q RoPE part, 16 KB
+constexpr int RBOX_BYTES = BN * 32 * 2;               // 64 keys x 32 RoPE dims, 4 KB
+constexpr int STAGE_BYTES = LAT_BYTES + RBOX_BYTES;   // bytes one stage's loads bring
+// Shared-memory K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half,
+// 128-byte swizzle) of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage
+// s (64-byte swizzle) at OFF_KVR + s * RBOX_BYTES.  Stages 2i and 2i+1 are adjacent
+// within every box column, so one N=128 score MMA covers two consecutive 64-key blocks.
+constexpr int QR_BYTES = TM * 32 * 2;                 // this CTA's Q RoPE part, 8 KB
 constexpr int X_BYTES = TM * BN * 2;                  // exchange buffer, 16 KB: the peer's
                                                       // partial scores as fp16, chunk-major
-                                                      // [8 x 16 B][128 rows]; then P
-                                                      // (bf16, 128-byte swizzled rows)
+                                                      // [8 x 16 B][128 rows]
+constexpr int P_BYTES = TM * BN * 2;                  // P, bf16, 128-byte swizzled rows
 constexpr int NTHREADS = 320;
 
 constexpr int OFF_KV = 0;
 constexpr int OFF_KVR = OFF_KV + NST * LAT_BYTES;
-constexpr int OFF_QR = OFF_KV + NST * STAGE_BYTES;
-constexpr int OFF_X = OFF_QR + QR_BYTES;              // [2] exchange / P buffers
-constexpr int OFF_M = OFF_X + 2 * X_BYTES;            // running max handoff [2][128]
+constexpr int OFF_QR = OFF_KVR + NST * RBOX_BYTES;
+constexpr int OFF_X = OFF_QR + QR_BYTES;              // [2] exchange buffers
+constexpr int OFF_P = OFF_X + 2 * X_BYTES;            // [2] P buffers
+constexpr int OFF_M = OFF_P + 2 * P_BYTES;            // running max handoff [2][128]
 constexpr int OFF_L = OFF_M + 2 * TM * 4;             // final (l, m) per warpgroup [2][2][128]
 constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
 
@@ -73,7 +73,7 @@ enum {
   B_SF,                     // S buffer full (MMA commit)                  [2]
   B_SE = B_SF + 2,          // S buffer read (128 threads)                 [2]
   B_XF = B_SE + 2,          // peer's partial scores landed (tx bytes)     [2]
-  B_XE = B_XF + 2,          // peer's PV done with its buffer (1 remote)   [2]
+  B_XE = B_XF + 2,          // peer read the scores sent it (1 remote)    [2]
   B_PF = B_XE + 2,          // P complete, O rescaled (128)                [2]
   B_PE = B_PF + 2,          // PV done (MMA commit)                        [2]
   B_M = B_PE + 2,           // running max of a block published (128)      [2]
@@ -131,8 +131,8 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-    attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                  AttnArgs a) {
+    attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
+                  const __grid_constant__ CUtensorMap tmQR, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -199,12 +199,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
-      if (rank == 1) {
-        prefetch_tmap(&tmQ);
-        mbar_expect_tx(&bar[B_QR], QR_BYTES);
-        tma_load_2d(sm + OFF_QR, &tmQ, &bar[B_QR], G.Dc, (int32_t)grow0);
-      }
-      const uint32_t bytes = rank == 1 ? STAGE_BYTES : LAT_BYTES;
+      prefetch_tmap(&tmKR);
+      prefetch_tmap(&tmQR);
+      mbar_expect_tx(&bar[B_QR], QR_BYTES);
+      tma_load_2d(sm + OFF_QR, &tmQR, &bar[B_QR], G.Dc + (int)rank * 32, (int32_t)grow0);
+      const uint32_t bytes = STAGE_BYTES;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NST;
         if (!mbar_wait(&bar[B_KVE + s], ((j / NST) & 1) ^ 1, abort, a.err, 0x101, j)) break;
@@ -216,9 +215,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int q = 0; q < 4; ++q)
           tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
                       (int)rank * HALF + q * 64, (int32_t)slot0, b);
-        if (rank == 1)
-          tma_load_3d(sm + OFF_KVR + s * BOX_BYTES, &tmK, &bar[B_KVF + s], G.Dc,
-                      (int32_t)slot0, b);
+        tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s], G.Dc + (int)rank * 32,
+                    (int32_t)slot0, b);
       }
     }
   } else if (warp == 9) {
@@ -232,7 +230,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const uint32_t id_qk = idesc_bf16(128, 2 * BN, false, false);
       const uint32_t id_pv = idesc_bf16(128, HALF, false, true);
       bool ok = mbar_wait(&bar[B_QREADY], 0, abort, a.err, 0x102, 0);
-      if (ok && rank == 1) ok = mbar_wait(&bar[B_QR], 0, abort, a.err, 0x103, 0);
+      if (ok) ok = mbar_wait(&bar[B_QR], 0, abort, a.err, 0x103, 0);
       tc_fence_after();
       int next_pv = 0;                         // next block whose PV is to be issued
       auto issue_pv = [&](int jj) {
@@ -240,7 +238,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int s = jj % NST;
         tc_fence_after();
         const uint32_t v0 = smem_u32(sm + OFF_KV + s * BOX_BYTES);
-        const uint32_t pa = smem_u32(sm + OFF_X + pb * X_BYTES);
+        const uint32_t pa = smem_u32(sm + OFF_P + pb * P_BYTES);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
@@ -248,9 +246,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                  (jj > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bar[B_PE + pb]);
         mma_commit(&bar[B_KVE + s]);
-        // the peer's warpgroup waits for this before refilling the buffer at block jj+2;
-        // no signal is sent that nobody waits for (the peer may have exited by then)
-        if (jj + 2 < nblk) mma_commit_cluster(&bar[B_XE + pb], (uint16_t)(1u << peer));
       };
       // issue every PV whose P is ready, for blocks below `limit`, without blocking
       auto pv_ready = [&](int limit) {
@@ -291,21 +286,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (!wait_pv(&bar[B_SE + 1], ph, j0, 0x106, j0 + 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + S_COL;
-        const uint32_t k0 = smem_u32(sm + OFF_KV + s0 * BOX_BYTES);
+        // descriptor of K box column 0 at stage s0; the 16-dim steps only add offsets
+        const uint64_t kd = desc_sw128(smem_u32(sm + OFF_KV + s0 * BOX_BYTES), 16, 1024);
+        mma_ts(d, tmem + Q_COL, kd, id_qk, 0u);
 #pragma unroll
-        for (int kk = 0; kk < HALF / 16; ++kk) {
+        for (int kk = 1; kk < HALF / 16; ++kk)
           mma_ts(d, tmem + Q_COL + kk * 8,
-                 desc_sw128(k0 + (kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32, 16, 1024), id_qk,
-                 kk > 0 ? 1u : 0u);
-        }
-        if (rank == 1) {
-          const uint32_t qa = smem_u32(sm + OFF_QR);
-          const uint32_t kr = smem_u32(sm + OFF_KVR + s0 * BOX_BYTES);
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            mma_ss(d, desc_sw128(qa + w * 32, 16, 1024), desc_sw128(kr + w * 32, 16, 1024),
-                   id_qk, 1u);
-        }
+                 kd + (uint64_t)(((kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32) >> 4), id_qk, 1u);
+        const uint64_t qd = desc_sw64(smem_u32(sm + OFF_QR), 512);
+        const uint64_t rd = desc_sw64(smem_u32(sm + OFF_KVR + s0 * RBOX_BYTES), 512);
+        mma_ss(d, qd, rd, id_qk, 1u);
+        mma_ss(d, qd + 2, rd + 2, id_qk, 1u);           // second 16-dim step: +32 bytes
         mma_commit(&bar[B_SF]);
         mma_commit(&bar[B_SF + 1]);
         pv_ready(j0);
@@ -357,7 +348,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * X_BYTES), peer) + (uint32_t)t * 16;
     const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
     const uint4* my_x = reinterpret_cast<const uint4*>(sm + OFF_X + wg * X_BYTES) + t;
-    uint8_t* prow = sm + OFF_X + wg * X_BYTES + t * 128;     // P row t over the same buffer
+    uint8_t* prow = sm + OFF_P + wg * P_BYTES + t * 128;     // P row t
+    const uint32_t peer_xe = mapa(smem_u32(&bar[B_XE + wg]), peer);
     const float c2 = a.scale_log2;
     float m_last = -INFINITY, l = 0.f;         // this warpgroup's running sum and its max
     bool ok = true;
@@ -442,7 +434,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           s[8 * q + 2 * e + 1] += f.y;
         }
       }
-      named_bar(1 + wg, TM);            // the whole buffer is read before P overwrites it
+      named_bar(1 + wg, TM);            // the whole buffer is read: hand it back
+      if (t == 0) mbar_arrive_cluster(peer_xe);
 
       // masked raw maximum (scores are scaled inside the exponent)
       const int64_t lim64 = k_end_row - g0;
@@ -488,12 +481,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       l = l * ex2(m_last - msub) + sum;
       m_last = m;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-
-      // warp-collective TMEM access: the whole warp rescales O if any of its rows grew
+      // P buffer of this warpgroup is free once PV of its previous block has finished;
+      // O is rescaled (warp-collective TMEM access) after PV of the previous block
       if (j > 0 && __any_sync(FULL, fac != 1.f)) {
         if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
                                         a.err, 0x205, (t << 16) | j))) {
@@ -502,7 +491,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_after();
         rescale_row(tmem + lane_base + O_COL, fac);
+      } else if (j >= 2) {
+        if (!__all_sync(FULL, mbar_wait(&bar[B_PE + wg], kph ^ 1, abort, a.err, 0x206,
+                                        (t << 16) | j))) {
+          ok = false;
+          break;
+        }
       }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar[B_PF + wg]);
@@ -560,18 +559,20 @@ bool tc_attend_supported(const Geo& g) { return g.Dc == 2 * HALF && g.Dr == 64; 
 cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
                       const void* cache, int64_t k_first, int64_t n_keys, float scale,
                       void* o_lat, float* lse, unsigned int* err, cudaStream_t st) {
-  CUtensorMap K, Q;
+  CUtensorMap K, KR, QR;
   {
     uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.S, (uint64_t)g.B};
     uint64_t s[2] = {(uint64_t)g.row * 2, (uint64_t)g.S * g.row * 2};
     uint32_t b[3] = {64, BN, 1};
     if (!make_tmap_bf16(&K, cache, 3, d, s, b)) return cudaErrorInvalidValue;
+    uint32_t br[3] = {32, BN, 1};
+    if (!make_tmap_bf16(&KR, cache, 3, d, s, br, true)) return cudaErrorInvalidValue;
   }
   {
     uint64_t d[2] = {(uint64_t)g.row, (uint64_t)g.B * n_q * g.H};
     uint64_t s[1] = {(uint64_t)g.row * 2};
-    uint32_t b[2] = {64, TM};
-    if (!make_tmap_bf16(&Q, q_abs, 2, d, s, b)) return cudaErrorInvalidValue;
+    uint32_t b[2] = {32, TM};
+    if (!make_tmap_bf16(&QR, q_abs, 2, d, s, b, true)) return cudaErrorInvalidValue;
   }
   static bool attr = false;
   if (!attr) {
@@ -590,7 +591,7 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
   a.err = err;
   const int64_t tiles = (int64_t)g.B * a.tiles_per_batch;
-  attend_kernel<<<(unsigned)(2 * tiles), NTHREADS, ATT_SMEM, st>>>(K, Q, a);
+  attend_kernel<<<(unsigned)(2 * tiles), NTHREADS, ATT_SMEM, st>>>(K, KR, QR, a);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;

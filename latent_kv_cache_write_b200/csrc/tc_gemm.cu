@@ -223,12 +223,27 @@ __global__ void __launch_bounds__(GTHREADS, 1)
           // q_abs[.., Dc:] = RoPE(q_R) for this tile's rows and head
           const int64_t i = m % p.rows_per_batch;
           const int64_t g = p.first_tok + i;
-          const bf16* src = p.q_rope + (m * G.H + z) * G.Dr;
-          bf16* dst = p.out + (m * G.H + z) * G.row + G.Dc;
-          for (int q = 0; q < G.Dr / 2; ++q) {
-            float a = __bfloat162float(src[2 * q]), b = __bfloat162float(src[2 * q + 1]);
-            rope_rotate_fast(a, b, (double)rope_pos(G, g, q), inv_freq[q]);
-            *reinterpret_cast<uint32_t*>(dst + 2 * q) = pack_bf16(a, b);
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + (m * G.H + z) * G.Dr);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (m * G.H + z) * G.row + G.Dc);
+          // 8 bf16 (4 pairs) per 16-byte vector; the loads of a chunk are issued together
+          for (int c = 0; c < G.Dr / 8; c += 4) {
+            uint4 in[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) in[u] = c + u < G.Dr / 8 ? src[c + u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (c + u >= G.Dr / 8) break;
+              uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int q = (c + u) * 4 + e;
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                float a = f.x, b = f.y;
+                rope_rotate_fast(a, b, (double)rope_pos(G, g, q), inv_freq[q]);
+                w[e] = pack_bf16(a, b);
+              }
+              dst[c + u] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
       }

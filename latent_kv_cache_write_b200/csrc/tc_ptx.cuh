@@ -6,7 +6,7 @@
 //   [0,14)  start address >> 4        [16,30) leading byte offset >> 4
 //   [32,46) stride byte offset >> 4   [46,48) version = 1
 //   [49,52) base offset = 0           [52]    LBO mode = 0
-//   [61,64) swizzle: 2 = 128-byte swizzle
+//   [61,64) swizzle: 2 = 128-byte swizzle, 4 = 64-byte swizzle
 // A 128-byte-swizzled tile is made of 1024-byte atoms of 8 rows x 128 bytes; the 16-byte
 // chunk c of row r sits at chunk position c ^ (r % 8).  K-major: rows are M/N indices,
 // the 64 bf16 of a row run along K; SBO = distance between 8-row groups.  MN-major: rows
@@ -183,6 +183,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Arrive (relaxed, cluster scope) on a barrier given by its shared::cluster address: for
+// credits whose protected reads have already completed (their values are in registers).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
@@ -291,6 +298,12 @@ __device__ __forceinline__ void tmem_wait_st() {
 __host__ __device__ constexpr uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// 64-byte swizzled K-major tile: atoms of 8 rows x 64 bytes (SBO = 512 for packed rows).
+__host__ __device__ constexpr uint64_t desc_sw64(uint32_t saddr, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
 }
 
 // kind::f16, bf16 x bf16 -> f32

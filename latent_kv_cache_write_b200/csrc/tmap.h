@@ -9,9 +9,9 @@
 namespace mla {
 
 // bf16 tensor of `rank` dims (dims[0] contiguous), strides in bytes for dims 1..rank-1,
-// box in elements, 128-byte swizzle, out-of-bounds elements read as zero.
-// Returns false if the driver rejects the description.
+// box in elements, 128-byte swizzle (64-byte when swizzle64), out-of-bounds elements
+// read as zero.  Returns false if the driver rejects the description.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box);
+                    const uint64_t* strides_bytes, const uint32_t* box, bool swizzle64 = false);
 
 }  // namespace mla

@@ -435,7 +435,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       }
       named_bar(1 + wg, TM);            // the whole buffer is read: hand it back
-      if (t == 0) mbar_arrive_cluster(peer_xe);
+      if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);
 
       // masked raw maximum (scores are scaled inside the exponent)
       const int64_t lim64 = k_end_row - g0;

@@ -118,8 +118,10 @@ mla_status mla_absorb_q(const mla_shape* shape, const void* q_nope, const void* 
                         void* stream);
 
 /*
- * mla_attend_workspace_size — bytes of device workspace mla_attend needs for this
- * problem (split-key partial results and their log-sum-exps).  May be 0.
+ * mla_attend_workspace_size — bytes of device workspace that lets mla_attend split the
+ * key range of a tile across SMs (split-key partial outputs, float32, and their
+ * log-sum-exps, two slots per resident cluster of the current device).  May be 0 (the
+ * float32 path, and shapes without the tensor-core kernel, never need one).
  */
 size_t mla_attend_workspace_size(const mla_shape* shape, int64_t n_q, int64_t n_keys);
 
@@ -141,12 +143,16 @@ size_t mla_attend_workspace_size(const mla_shape* shape, int64_t n_q, int64_t n_
  *   cache  [B, S, d_latent + d_rope]          read
  *   o_lat  [B, n_q, n_h, d_latent]            written
  *   lse    [B, n_q, n_h] float32 or NULL      written
- *   workspace: device scratch of at least mla_attend_workspace_size() bytes (may be
- *   NULL when that size is 0); its contents on entry do not matter.
+ *   workspace: device scratch of at least mla_attend_workspace_size() bytes, or NULL
+ *   with workspace_bytes 0; its contents on entry do not matter.  Without it the work
+ *   is still spread over the SMs, but only in whole 128-row tiles (slower when there
+ *   are few tiles or they do not divide evenly).  Calls that share a workspace must
+ *   not run concurrently.
  * A single query per sequence (n_q == 1) is the decode case.
  * Errors: MLA_ERR_RANGE if n_keys > S, n_keys < 1, or the queries are not inside the
  * key window (k_first_tok <= q_first_tok and q_first_tok + n_q <= k_first_tok +
- * n_keys); MLA_ERR_ARG if workspace_bytes is too small.
+ * n_keys); MLA_ERR_ARG if a workspace is given (or workspace_bytes > 0) and it is
+ * NULL or smaller than mla_attend_workspace_size().
  */
 mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
                       int64_t q_first_tok, const void* cache, int64_t k_first_tok,

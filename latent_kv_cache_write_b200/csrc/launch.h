@@ -37,9 +37,14 @@ cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_
                     unsigned int* err, cudaStream_t st);
 
 bool tc_attend_supported(const Geo& g);
+// Workspace for split-key partials on the current device (0 if it cannot be queried).
+size_t tc_attend_workspace(const Geo& g);
+// With workspace_bytes >= tc_attend_workspace(g) tiles may be split across clusters;
+// otherwise (workspace may be null) the schedule cuts on tile boundaries only.
 cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
                       const void* cache, int64_t k_first, int64_t n_keys, float scale,
-                      void* o_lat, float* lse, unsigned int* err, cudaStream_t st);
+                      void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
+                      unsigned int* err, cudaStream_t st);
 
 // Device address of the library's error word on the current device (nullptr on failure).
 unsigned int* device_error_word();

@@ -130,7 +130,10 @@ mla_status mla_absorb_q(const mla_shape* shape, const void* q_nope, const void* 
 }
 
 size_t mla_attend_workspace_size(const mla_shape* shape, int64_t n_q, int64_t n_keys) {
-  (void)shape; (void)n_q; (void)n_keys;
+  (void)n_q; (void)n_keys;
+  Geo g;
+  if (check_shape(shape, &g) != MLA_OK) return 0;
+  if (shape->dtype == MLA_BF16 && tc_attend_supported(g)) return tc_attend_workspace(g);
   return 0;
 }
 
@@ -149,15 +152,18 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
   if (n_q > 65535) return MLA_ERR_UNSUPPORTED;
   if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(o_lat) || (lse && !aligned16(lse)))
     return MLA_ERR_ALIGN;
+  // no workspace at all is allowed (the schedule then keeps tiles whole); a workspace
+  // that is given must be large enough
   const size_t need = mla_attend_workspace_size(shape, n_q, n_keys);
-  if (workspace_bytes < need || (need > 0 && !workspace)) return MLA_ERR_ARG;
+  if ((workspace || workspace_bytes > 0) && (!workspace || workspace_bytes < need))
+    return MLA_ERR_ARG;
   if (workspace && !aligned16(workspace)) return MLA_ERR_ALIGN;
   if (n_q == 0) return MLA_OK;
   const bool bf = shape->dtype == MLA_BF16;
   if (bf && tc_attend_supported(g))
     return cuda_status(tc_attend(g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
-                                 softmax_scale, o_lat, lse, device_error_word(),
-                                 (cudaStream_t)stream));
+                                 softmax_scale, o_lat, lse, workspace, workspace_bytes,
+                                 device_error_word(), (cudaStream_t)stream));
   return cuda_status(simt_attend(g, bf, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
                                  softmax_scale, o_lat, lse, (cudaStream_t)stream));
 }

@@ -24,13 +24,25 @@
 // units).  Masking is frame-block-causal per row; a ring that wraps is walked as two
 // contiguous slot segments.
 //
-// Warp roles (320 threads): warps 0-3 and 4-7 are the two softmax warpgroups (thread =
-// row = TMEM lane), warp 8 is the TMA producer, warp 9 the MMA issuer and TMEM owner.
+// Scheduling is persistent and split-key ("stream-K"): the launch has one cluster per
+// pair of SMs, and the key blocks of all tiles, laid end to end, are cut into one equal
+// range per cluster.  A cluster walks its range as segments (blocks [jb, je) of one
+// tile); a segment that covers its whole tile writes the final output, any other writes
+// its normalised partial output and log-sum-exp to the workspace, and a combine kernel
+// merges the partials of each split tile.  Without a workspace the cuts fall on tile
+// boundaries only.
+//
+// Warp roles (352 threads): warps 0-3 and 4-7 are the two softmax warpgroups (thread =
+// row = TMEM lane), warp 8 is the TMA producer, warp 9 issues the score MMAs, loads the
+// Q RoPE tiles and owns the TMEM allocation, warp 10 issues the PV MMAs.
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tmap.h"
 
 #include <cuda_fp16.h>
+
+#include <mutex>
+#include <vector>
 
 namespace mla {
 namespace {
@@ -47,14 +59,16 @@ constexpr int RBOX_BYTES = BN * 32 * 2;               // 64 keys x 32 RoPE dims,
 constexpr int STAGE_BYTES = LAT_BYTES + RBOX_BYTES;   // bytes one stage's loads bring
 // Shared-memory K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half,
 // 128-byte swizzle) of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage
-// s (64-byte swizzle) at OFF_KVR + s * RBOX_BYTES.  Stages 2i and 2i+1 are adjacent
-// within every box column, so one N=128 score MMA covers two consecutive 64-key blocks.
+// s (64-byte swizzle) at OFF_KVR + s * RBOX_BYTES.  Consecutive stages are adjacent
+// within every box column, so one N=128 score MMA covers two consecutive 64-key blocks
+// unless their stages wrap around the ring.
 constexpr int QR_BYTES = TM * 32 * 2;                 // this CTA's Q RoPE part, 8 KB
 constexpr int X_BYTES = TM * BN * 2;                  // exchange buffer, 16 KB: the peer's
                                                       // partial scores as fp16, chunk-major
                                                       // [8 x 16 B][128 rows]
 constexpr int P_BYTES = TM * BN * 2;                  // P, bf16, 128-byte swizzled rows
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 352;
+constexpr int MAXC = 128;                             // clusters one launch can schedule
 
 constexpr int OFF_KV = 0;
 constexpr int OFF_KVR = OFF_KV + NST * LAT_BYTES;
@@ -65,11 +79,16 @@ constexpr int OFF_M = OFF_P + 2 * P_BYTES;            // running max handoff [2]
 constexpr int OFF_L = OFF_M + 2 * TM * 4;             // final (l, m) per warpgroup [2][2][128]
 constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
 
+// A per-block barrier completes once per use of its buffer, a per-segment one once per
+// segment; a waiter counts the uses and waits on the parity of the count.
 enum {
   B_KVF = 0,                // K/V stage loaded (TMA)
   B_KVE = B_KVF + NST,      // K/V stage free (MMA commit after PV)
-  B_QR = B_KVE + NST,       // Q RoPE tile loaded
-  B_QREADY,                 // Q latent half written to TMEM (256 threads)
+  B_QR = B_KVE + NST,       // Q RoPE tile of a segment loaded (TMA)
+  B_QREADY,                 // Q latent half of a segment in TMEM (256 threads)
+  B_QKDONE,                 // every score MMA of a segment finished (MMA commit)
+  B_SEGDONE,                // every PV MMA of a segment finished (MMA commit)
+  B_OFREE,                  // O of a segment read out of TMEM (256 threads)
   B_SF,                     // S buffer full (MMA commit)                  [2]
   B_SE = B_SF + 2,          // S buffer read (128 threads)                 [2]
   B_XF = B_SE + 2,          // peer's partial scores landed (tx bytes)     [2]
@@ -77,11 +96,11 @@ enum {
   B_PF = B_XE + 2,          // P complete, O rescaled (128)                [2]
   B_PE = B_PF + 2,          // PV done (MMA commit)                        [2]
   B_M = B_PE + 2,           // running max of a block published (128)      [2]
-  B_DONE = B_M + 2,         // every MMA finished
-  NBAR
+  NBAR = B_M + 2
 };
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int ATT_SMEM = OFF_MISC + 16 + 1024;
+static_assert(ATT_SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
 
 constexpr uint32_t O_COL = 0, Q_COL = 256, S_COL = 384;
 constexpr unsigned FULL = 0xffffffffu;
@@ -93,10 +112,23 @@ struct AttnArgs {
   const bf16* q_abs;
   bf16* o_lat;
   float* lse;
+  float* ws_o;              // partial outputs [slot][TM][Dc], fp32, normalised by their l
+  float* ws_lse;            // their natural log-sum-exps [slot][TM]
   int tiles_per_batch;
   unsigned int* err;
 };
 
+// Cluster c walks the key blocks from (cut_tile[c], cut_blk[c]) up to, not including,
+// (cut_tile[c + 1], cut_blk[c + 1]) in tile-major order; its partial segments take the
+// workspace slots slot0[c], slot0[c] + 1, ...
+struct Sched {
+  int32_t cut_tile[MAXC + 1];
+  int32_t cut_blk[MAXC + 1];
+  int32_t slot0[MAXC];
+};
+
+// Key blocks of one tile: its rows see the keys k_first .. k_first + L - 1 (frame-
+// block-causal bound of its last row), stored in the ring as two contiguous slot runs.
 struct Blocks {
   int64_t k_first, p1, n1, L;
   int nb1, nblk;
@@ -117,6 +149,82 @@ struct Blocks {
   }
 };
 
+struct TileGeo {
+  int b;
+  int64_t rows_b, row0, grow0, i_last;
+  Blocks blk;
+};
+
+// one past the last key query i sees (frame-block-causal, clipped to the key window)
+__host__ __device__ inline int64_t key_end(const Geo& G, int64_t q_first, int64_t k_lim,
+                                           int64_t i) {
+  const int64_t e = ((q_first + i) / G.F + 1) * G.F;
+  return e < k_lim ? e : k_lim;
+}
+
+__host__ __device__ inline TileGeo tile_geo(const Geo& G, int64_t n_q, int64_t q_first,
+                                            int64_t k_first, int64_t n_keys,
+                                            int tiles_per_batch, int tile) {
+  TileGeo t;
+  t.b = tile / tiles_per_batch;
+  const int tb = tile - t.b * tiles_per_batch;
+  t.rows_b = n_q * G.H;
+  t.row0 = (int64_t)tb * TM;
+  t.grow0 = (int64_t)t.b * t.rows_b + t.row0;
+  const int64_t last_row = (t.row0 + TM < t.rows_b ? t.row0 + TM : t.rows_b) - 1;
+  t.i_last = last_row / G.H;
+  Blocks& k = t.blk;
+  k.k_first = k_first;
+  k.L = key_end(G, q_first, k_first + n_keys, t.i_last) - k_first;
+  k.p1 = k_first % G.S;
+  k.n1 = k.L < G.S - k.p1 ? k.L : G.S - k.p1;
+  k.nb1 = (int)((k.n1 + BN - 1) / BN);
+  k.nblk = k.nb1 + (int)((k.L - k.n1 + BN - 1) / BN);
+  return t;
+}
+
+// The segments of one cluster's range, in order.  Every role walks the same sequence
+// and keeps the running counts that barrier phases and ring stages derive from.
+struct SegWalk {
+  int tile, jb, je, tend, bend;
+  int k;                    // segment index within this cluster
+  int gbase;                // blocks of earlier segments (K/V ring position)
+  int nbase[2];             // blocks of earlier segments taken by each warpgroup
+  int slot;                 // workspace slot of the next partial segment
+  TileGeo tg;
+
+  __device__ void begin(const Sched& sc, const AttnArgs& a, int c) {
+    tile = sc.cut_tile[c];
+    jb = sc.cut_blk[c];
+    tend = sc.cut_tile[c + 1];
+    bend = sc.cut_blk[c + 1];
+    k = 0;
+    gbase = 0;
+    nbase[0] = nbase[1] = 0;
+    slot = sc.slot0[c];
+    load(a);
+  }
+  __device__ bool valid() const { return tile < tend || (tile == tend && jb < bend); }
+  __device__ void load(const AttnArgs& a) {
+    if (!valid()) return;
+    tg = tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, tile);
+    je = tile == tend ? bend : tg.blk.nblk;
+  }
+  __device__ int nb() const { return je - jb; }
+  __device__ bool partial() const { return jb > 0 || je < tg.blk.nblk; }
+  __device__ void next(const AttnArgs& a) {
+    const int n = nb();
+    gbase += n;
+    nbase[0] += (n + 1) >> 1;
+    nbase[1] += n >> 1;
+    if (partial()) ++slot;
+    ++k;
+    ++tile;
+    jb = 0;
+    load(a);
+  }
+};
+
 __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
 #pragma unroll 1
   for (int c = 0; c < HALF; c += 16) {
@@ -130,9 +238,29 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
+// Q latent half of row `grow` -> TMEM columns from `tq` (A operand of the score MMA),
+// bf16 pairs per column; each warpgroup loads half of the row.
+__device__ __forceinline__ void load_q(const AttnArgs& a, uint32_t tq, int64_t grow,
+                                       bool row_ok, uint32_t rank, int wg) {
+  const uint4* src = reinterpret_cast<const uint4*>(a.q_abs + grow * a.g.row + rank * HALF +
+                                                    wg * (HALF / 2));
+#pragma unroll 1
+  for (int c = 0; c < HALF / 64; ++c) {
+    uint32_t v[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 x = row_ok ? src[c * 4 + q] : make_uint4(0, 0, 0, 0);
+      v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+    }
+    tmem_st16(tq + wg * (HALF / 4) + c * 16, v);
+  }
+  tmem_wait_st();
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
-                  const __grid_constant__ CUtensorMap tmQR, AttnArgs a) {
+                  const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ AttnArgs a,
+                  const __grid_constant__ Sched sc) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -144,27 +272,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const uint32_t peer = rank ^ 1u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Geo& G = a.g;
-  const int tile = blockIdx.x >> 1;
-  const int b = tile / a.tiles_per_batch;
-  const int tb = tile - b * a.tiles_per_batch;
-  const int64_t rows_b = a.n_q * G.H;
-  const int64_t row0 = (int64_t)tb * TM;
-  const int64_t grow0 = (int64_t)b * rows_b + row0;
-  const int64_t k_lim = a.k_first + a.n_keys;
-  auto k_end_of = [&](int64_t i) {
-    const int64_t e = ((a.q_first + i) / G.F + 1) * G.F;
-    return e < k_lim ? e : k_lim;
-  };
-  const int64_t last_row = (row0 + TM < rows_b ? row0 + TM : rows_b) - 1;
-  const int64_t i_last = last_row / G.H;
-  Blocks blk;
-  blk.k_first = a.k_first;
-  blk.L = k_end_of(i_last) - a.k_first;
-  blk.p1 = a.k_first % G.S;
-  blk.n1 = blk.L < G.S - blk.p1 ? blk.L : G.S - blk.p1;
-  blk.nb1 = (int)((blk.n1 + BN - 1) / BN);
-  blk.nblk = blk.nb1 + (int)((blk.L - blk.n1 + BN - 1) / BN);
-  const int nblk = blk.nblk;
 
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -173,6 +280,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(&bar[B_QR], 1);
     mbar_init(&bar[B_QREADY], 256);
+    mbar_init(&bar[B_QKDONE], 1);
+    mbar_init(&bar[B_SEGDONE], 1);
+    mbar_init(&bar[B_OFREE], 256);
     for (int q = 0; q < 2; ++q) {
       mbar_init(&bar[B_SF + q], 1);
       mbar_init(&bar[B_SE + q], 128);
@@ -182,7 +292,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bar[B_PE + q], 1);
       mbar_init(&bar[B_M + q], 128);
     }
-    mbar_init(&bar[B_DONE], 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -195,348 +304,375 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  SegWalk sw;
+  sw.begin(sc, a, blockIdx.x >> 1);
+
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmKR);
-      prefetch_tmap(&tmQR);
-      mbar_expect_tx(&bar[B_QR], QR_BYTES);
-      tma_load_2d(sm + OFF_QR, &tmQR, &bar[B_QR], G.Dc + (int)rank * 32, (int32_t)grow0);
-      const uint32_t bytes = STAGE_BYTES;
-      for (int j = 0; j < nblk; ++j) {
-        const int s = j % NST;
-        if (!mbar_wait(&bar[B_KVE + s], ((j / NST) & 1) ^ 1, abort, a.err, 0x101, j)) break;
-        int64_t slot0, g0;
-        int valid;
-        blk.get(j, slot0, g0, valid);
-        mbar_expect_tx(&bar[B_KVF + s], bytes);
+      bool ok = true;
+      for (; ok && sw.valid(); sw.next(a)) {
+        for (int j = sw.jb; j < sw.je; ++j) {
+          const int g = sw.gbase + (j - sw.jb);
+          const int s = g % NST;
+          ok = mbar_wait(&bar[B_KVE + s], ((g / NST) & 1) ^ 1, abort, a.err, 0x101, g);
+          if (!ok) break;
+          int64_t slot0, g0;
+          int valid;
+          sw.tg.blk.get(j, slot0, g0, valid);
+          mbar_expect_tx(&bar[B_KVF + s], STAGE_BYTES);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
-                      (int)rank * HALF + q * 64, (int32_t)slot0, b);
-        tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s], G.Dc + (int)rank * 32,
-                    (int32_t)slot0, b);
+          for (int q = 0; q < 4; ++q)
+            tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
+                        (int)rank * HALF + q * 64, (int32_t)slot0, sw.tg.b);
+          tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s],
+                      G.Dc + (int)rank * 32, (int32_t)slot0, sw.tg.b);
+        }
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    // Scores of blocks 2i and 2i+1 are one N=128 series (S buffers 0 and 1 are adjacent);
-    // a score series is issued as soon as its data and S buffers are ready, since the
-    // scores start the softmax chains.  PV products are issued in block order, as soon as
-    // their P is ready whenever the issuer would otherwise wait: that frees the K/V stage
-    // for the next load and the exchange buffer for the peer early.
+    // ------------------------------------------------------------ score MMA issuer
+    // Scores of blocks 2i and 2i+1 of a segment are one N=128 series (S buffers 0 and 1
+    // are adjacent) when their stages are adjacent, else two N=64 series; a series is
+    // issued as soon as its data and S buffers are ready: the scores start the softmax
+    // chains.  An MMA issue blocks while the tensor pipe is busy, so the PV products
+    // have their own issuing thread.  A segment's Q RoPE tile is loaded once every score
+    // MMA of the previous segment has finished.
     if (lane == 0) {
-      const uint32_t id_qk = idesc_bf16(128, 2 * BN, false, false);
-      const uint32_t id_pv = idesc_bf16(128, HALF, false, true);
-      bool ok = mbar_wait(&bar[B_QREADY], 0, abort, a.err, 0x102, 0);
-      if (ok) ok = mbar_wait(&bar[B_QR], 0, abort, a.err, 0x103, 0);
-      tc_fence_after();
-      int next_pv = 0;                         // next block whose PV is to be issued
-      auto issue_pv = [&](int jj) {
-        const int pb = jj & 1;
-        const int s = jj % NST;
-        tc_fence_after();
-        const uint32_t v0 = smem_u32(sm + OFF_KV + s * BOX_BYTES);
-        const uint32_t pa = smem_u32(sm + OFF_P + pb * P_BYTES);
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
-                 desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
-                 (jj > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar[B_PE + pb]);
-        mma_commit(&bar[B_KVE + s]);
-      };
-      // issue every PV whose P is ready, for blocks below `limit`, without blocking
-      auto pv_ready = [&](int limit) {
-        while (next_pv < limit &&
-               mbar_test_wait(&bar[B_PF + (next_pv & 1)], (next_pv >> 1) & 1)) {
-          issue_pv(next_pv);
-          ++next_pv;
-        }
-      };
-      // wait for a phase while keeping the PV stream moving
-      auto wait_pv = [&](uint64_t* w, uint32_t parity, int limit, uint32_t site, int j) -> bool {
-        if (mbar_test_wait(w, parity)) return true;
-        const long long c0 = clock64();
-        for (uint32_t it = 1;; ++it) {
-          pv_ready(limit);
-          if (mbar_test_wait(w, parity)) return true;
-          if ((it & 255u) == 0) {
-            if (*abort) return false;
-            if (clock64() - c0 > 4000000000ll) {
-              *abort = 1;
-              report_timeout(a.err, site, (uint32_t)j);
-              return false;
-            }
-          }
-        }
-      };
-      const int npair = (nblk + 1) / 2;
-      for (int i = 0; ok && i < npair; ++i) {
-        const int j0 = 2 * i, s0 = j0 % NST;
-        const bool two = j0 + 1 < nblk;
-        const uint32_t ph = (i & 1) ^ 1;
-        if (!wait_pv(&bar[B_KVF + s0], (j0 / NST) & 1, j0, 0x105, j0)) { ok = false; break; }
-        if (two && !wait_pv(&bar[B_KVF + s0 + 1], (j0 / NST) & 1, j0, 0x105, j0 + 1)) {
-          ok = false;
-          break;
-        }
-        if (!wait_pv(&bar[B_SE], ph, j0, 0x106, j0)) { ok = false; break; }
-        if (!wait_pv(&bar[B_SE + 1], ph, j0, 0x106, j0 + 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d = tmem + S_COL;
-        // descriptor of K box column 0 at stage s0; the 16-dim steps only add offsets
-        const uint64_t kd = desc_sw128(smem_u32(sm + OFF_KV + s0 * BOX_BYTES), 16, 1024);
-        mma_ts(d, tmem + Q_COL, kd, id_qk, 0u);
+      prefetch_tmap(&tmQR);
+      const uint32_t id_qk1 = idesc_bf16(128, BN, false, false);
+      // one score series: S columns [d, d + N) for the keys of stage s onwards
+      auto qk_series = [&](uint32_t d, int s, uint32_t id) {
+        // descriptor of K box column 0 at stage s; the 16-dim steps only add offsets
+        const uint64_t kd = desc_sw128(smem_u32(sm + OFF_KV + s * BOX_BYTES), 16, 1024);
+        mma_ts(d, tmem + Q_COL, kd, id, 0u);
 #pragma unroll
         for (int kk = 1; kk < HALF / 16; ++kk)
           mma_ts(d, tmem + Q_COL + kk * 8,
-                 kd + (uint64_t)(((kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32) >> 4), id_qk, 1u);
+                 kd + (uint64_t)(((kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32) >> 4), id, 1u);
         const uint64_t qd = desc_sw64(smem_u32(sm + OFF_QR), 512);
-        const uint64_t rd = desc_sw64(smem_u32(sm + OFF_KVR + s0 * RBOX_BYTES), 512);
-        mma_ss(d, qd, rd, id_qk, 1u);
-        mma_ss(d, qd + 2, rd + 2, id_qk, 1u);           // second 16-dim step: +32 bytes
-        mma_commit(&bar[B_SF]);
-        mma_commit(&bar[B_SF + 1]);
-        pv_ready(j0);
-      }
-      // remaining PV products
-      while (ok && next_pv < nblk) {
-        if (!mbar_wait(&bar[B_PF + (next_pv & 1)], (next_pv >> 1) & 1, abort, a.err, 0x104,
-                       next_pv)) {
-          ok = false;
-          break;
+        const uint64_t rd = desc_sw64(smem_u32(sm + OFF_KVR + s * RBOX_BYTES), 512);
+        mma_ss(d, qd, rd, id, 1u);
+        mma_ss(d, qd + 2, rd + 2, id, 1u);              // second 16-dim step: +32 bytes
+      };
+      bool ok = true;
+      for (; ok && sw.valid(); sw.next(a)) {
+        const uint32_t kph = sw.k & 1;
+        if (sw.k > 0) ok = mbar_wait(&bar[B_QKDONE], kph ^ 1, abort, a.err, 0x107, sw.k);
+        if (!ok) break;
+        mbar_expect_tx(&bar[B_QR], QR_BYTES);
+        tma_load_2d(sm + OFF_QR, &tmQR, &bar[B_QR], G.Dc + (int)rank * 32,
+                    (int32_t)sw.tg.grow0);
+        ok = mbar_wait(&bar[B_QREADY], kph, abort, a.err, 0x102, sw.k);
+        if (ok) ok = mbar_wait(&bar[B_QR], kph, abort, a.err, 0x103, sw.k);
+        if (!ok) break;
+        tc_fence_after();
+        const int n = sw.nb();
+        for (int jl = 0; jl < n; ++jl) {
+          const int w = jl & 1;                          // S buffer = warpgroup
+          const int g = sw.gbase + jl, s = g % NST;
+          const int q = sw.nbase[w] + (jl >> 1);         // S buffer use
+          ok = mbar_wait(&bar[B_KVF + s], (g / NST) & 1, abort, a.err, 0x105, g);
+          if (ok) ok = mbar_wait(&bar[B_SE + w], (q & 1) ^ 1, abort, a.err, 0x106, g);
+          if (!ok) break;
+          tc_fence_after();
+          qk_series(tmem + S_COL + w * BN, s, id_qk1);
+          mma_commit(&bar[B_SF + w]);
         }
-        issue_pv(next_pv);
-        ++next_pv;
+        mma_commit(&bar[B_QKDONE]);
       }
-      mma_commit(&bar[B_DONE]);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ PV issuer
+    // O += P . V in block order as each P is ready; the commits free the K/V stage for
+    // the next load and the P buffer, and let the softmax rescale O.  A segment starts
+    // once the previous segment's O has been read out (its first PV overwrites O); its
+    // last commit also covers its score MMAs: a block's P exists only after its scores
+    // were read.
+    if (lane == 0) {
+      const uint32_t id_pv = idesc_bf16(128, HALF, false, true);
+      bool ok = true;
+      for (; ok && sw.valid(); sw.next(a)) {
+        if (sw.k > 0) ok = mbar_wait(&bar[B_OFREE], (sw.k - 1) & 1, abort, a.err, 0x108, sw.k);
+        const int n = sw.nb();
+        for (int jl = 0; ok && jl < n; ++jl) {
+          const int pb = jl & 1, seq = sw.nbase[pb] + (jl >> 1);
+          const int g = sw.gbase + jl, s = g % NST;
+          ok = mbar_wait(&bar[B_PF + pb], seq & 1, abort, a.err, 0x104, g);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(sm + OFF_KV + s * BOX_BYTES);
+          const uint32_t pa = smem_u32(sm + OFF_P + pb * P_BYTES);
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
+                   desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
+                   (jl > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar[B_PE + pb]);
+          mma_commit(&bar[B_KVE + s]);
+        }
+        if (ok) mma_commit(&bar[B_SEGDONE]);
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
     const int wg = warp >> 2;                  // warpgroup: even (0) or odd (1) blocks
     const int t = tid & (TM - 1);              // row of the tile == TMEM lane
-    const int64_t r_in_b = row0 + t;
-    const bool row_valid = r_in_b < rows_b;
-    const int64_t grow = grow0 + t;
-    const int64_t k_end_row = k_end_of(row_valid ? r_in_b / G.H : i_last);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     float* m_sh = reinterpret_cast<float*>(sm + OFF_M);
     float* l_sh = reinterpret_cast<float*>(sm + OFF_L);
-
-    // Q latent half -> TMEM (A operand of the score MMA), bf16 pairs per column; each
-    // warpgroup loads half of the row
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(a.q_abs + grow * G.row + rank * HALF +
-                                                        wg * (HALF / 2));
-#pragma unroll 1
-      for (int c = 0; c < HALF / 64; ++c) {
-        uint32_t v[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 x = row_valid ? src[c * 4 + q] : make_uint4(0, 0, 0, 0);
-          v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
-        }
-        tmem_st16(tmem + lane_base + Q_COL + wg * (HALF / 4) + c * 16, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar[B_QREADY]);
-    }
-
     const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * X_BYTES), peer) + (uint32_t)t * 16;
     const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
     const uint4* my_x = reinterpret_cast<const uint4*>(sm + OFF_X + wg * X_BYTES) + t;
     uint8_t* prow = sm + OFF_P + wg * P_BYTES + t * 128;     // P row t
     const uint32_t peer_xe = mapa(smem_u32(&bar[B_XE + wg]), peer);
     const float c2 = a.scale_log2;
-    float m_last = -INFINITY, l = 0.f;         // this warpgroup's running sum and its max
     bool ok = true;
-    for (int j = wg; j < nblk; j += 2) {
-      const uint32_t kph = (j >> 1) & 1;
-      // arm this block's exchange: the peer's asynchronous stores complete X_BYTES of
-      // transactions on it (they may land before or after this arrive)
-      if (t == 0) mbar_expect_tx(&bar[B_XF + wg], X_BYTES);
-      if (!__all_sync(FULL, mbar_wait(&bar[B_SF + wg], kph, abort, a.err, 0x201, (t << 16) | j))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[64];
-      {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + S_COL + wg * BN, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(v[c]);
-        tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(v[c]);
-      }
+
+    if (sw.valid()) {
+      load_q(a, tmem + lane_base + Q_COL, sw.tg.grow0 + t, sw.tg.row0 + t < sw.tg.rows_b, rank,
+             wg);
       tc_fence_before();
-      mbar_arrive(&bar[B_SE + wg]);
-
-      // send this CTA's partial scores into the peer's buffer once the peer's PV of two
-      // blocks ago no longer reads it
-      if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], kph ^ 1, abort, a.err, 0x202,
-                                               (t << 16) | j))) {
-        ok = false;
-        break;
-      }
-      // both CTAs add the same two fp16-rounded partials, so their softmax agrees bit
-      // for bit; the rounding is ~2^-11 of a partial score
-      uint32_t hs[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        __half2 h2 = __floats2half2_rn(s[2 * c], s[2 * c + 1]);
-        hs[c] = *reinterpret_cast<uint32_t*>(&h2);
-        const float2 back = __half22float2(h2);
-        s[2 * c] = back.x;
-        s[2 * c + 1] = back.y;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        st_async_v4(peer_x + q * (TM * 16), hs[4 * q], hs[4 * q + 1], hs[4 * q + 2],
-                    hs[4 * q + 3], peer_xf);
-
-      int64_t slot0, g0;
-      int valid;
-      blk.get(j, slot0, g0, valid);
-      if (valid < BN && t < BN && t >= valid) {
-        // a partial block: zero this CTA's latent rows past the last key so that masked
-        // keys contribute exact zeros to P.V whatever the ring holds there (the stage has
-        // landed: QK of this block has completed)
-        uint8_t* st = sm + OFF_KV + (j % NST) * BOX_BYTES + t * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4* p = reinterpret_cast<uint4*>(st + q * NST * BOX_BYTES);
-#pragma unroll
-          for (int w = 0; w < 8; ++w) p[w] = make_uint4(0, 0, 0, 0);
-        }
-      }
-
-      // full scores: add the peer's partial
-      if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + wg], kph, abort, a.err, 0x203,
-                                               (t << 16) | j))) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 x = my_x[q * TM];
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-          s[8 * q + 2 * e] += f.x;
-          s[8 * q + 2 * e + 1] += f.y;
-        }
-      }
-      named_bar(1 + wg, TM);            // the whole buffer is read: hand it back
-      if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);
-
-      // masked raw maximum (scores are scaled inside the exponent)
-      const int64_t lim64 = k_end_row - g0;
-      const int lim = lim64 < valid ? (lim64 < 0 ? 0 : (int)lim64) : valid;
-      if (lim < BN) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = c < lim ? s[c] : -INFINITY;
-      }
-      float rmax = s[0];
-#pragma unroll
-      for (int c = 1; c < 64; ++c) rmax = fmaxf(rmax, s[c]);
-      const float mb = rmax * c2;
-
-      // running maximum after the previous block (published by the other warpgroup)
-      float m_prev = -INFINITY;
-      if (j > 0) {
-        if (!__all_sync(FULL, mbar_wait(&bar[B_M + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
-                                        a.err, 0x204, (t << 16) | j))) {
-          ok = false;
-          break;
-        }
-        m_prev = m_sh[((j - 1) & 1) * TM + t];
-      }
-      float m = m_prev, fac = 1.f;
-      if (j == 0) {
-        m = mb;
-      } else if (mb > m_prev + 8.f) {
-        m = mb;
-        fac = ex2(m_prev - m);
-      }
-      m_sh[wg * TM + t] = m;
-      mbar_arrive(&bar[B_M + wg]);
-
-      const float msub = m == -INFINITY ? 0.f : m;
-      uint32_t pk[32];
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2(fmaf(s[2 * c], c2, -msub));
-        const float p1 = ex2(fmaf(s[2 * c + 1], c2, -msub));
-        sum += p0 + p1;
-        pk[c] = pack_bf16(p0, p1);
-      }
-      l = l * ex2(m_last - msub) + sum;
-      m_last = m;
-      // P buffer of this warpgroup is free once PV of its previous block has finished;
-      // O is rescaled (warp-collective TMEM access) after PV of the previous block
-      if (j > 0 && __any_sync(FULL, fac != 1.f)) {
-        if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort,
-                                        a.err, 0x205, (t << 16) | j))) {
+      mbar_arrive(&bar[B_QREADY]);
+    }
+    for (; sw.valid(); sw.next(a)) {
+      const TileGeo& tg = sw.tg;
+      const int64_t r_in_b = tg.row0 + t;
+      const bool row_valid = r_in_b < tg.rows_b;
+      const int64_t grow = tg.grow0 + t;
+      const int64_t k_end_row =
+          key_end(G, a.q_first, a.k_first + a.n_keys, row_valid ? r_in_b / G.H : tg.i_last);
+      const int n = sw.nb();
+      float m_last = -INFINITY, l = 0.f;       // this warpgroup's running sum and its max
+      for (int jl = wg; jl < n; jl += 2) {
+        const int j = sw.jb + jl;              // block of the tile
+        const int seq = sw.nbase[wg] + (jl >> 1);
+        const uint32_t kph = seq & 1;
+        // arm this block's exchange: the peer's asynchronous stores complete X_BYTES of
+        // transactions on it (they may land before or after this arrive)
+        if (t == 0) mbar_expect_tx(&bar[B_XF + wg], X_BYTES);
+        if (!__all_sync(FULL, mbar_wait(&bar[B_SF + wg], kph, abort, a.err, 0x201, (t << 16) | j))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        rescale_row(tmem + lane_base + O_COL, fac);
-      } else if (j >= 2) {
+        float s[64];
+        {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + S_COL + wg * BN, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(v[c]);
+          tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(v[c]);
+        }
+        tc_fence_before();
+        mbar_arrive(&bar[B_SE + wg]);
+
+        // send this CTA's partial scores into the peer's buffer once the peer has read
+        // what was sent two blocks ago
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], kph ^ 1, abort, a.err, 0x202,
+                                                 (t << 16) | j))) {
+          ok = false;
+          break;
+        }
+        // both CTAs add the same two fp16-rounded partials, so their softmax agrees bit
+        // for bit; the rounding is ~2^-11 of a partial score
+        uint32_t hs[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          __half2 h2 = __floats2half2_rn(s[2 * c], s[2 * c + 1]);
+          hs[c] = *reinterpret_cast<uint32_t*>(&h2);
+          const float2 back = __half22float2(h2);
+          s[2 * c] = back.x;
+          s[2 * c + 1] = back.y;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_async_v4(peer_x + q * (TM * 16), hs[4 * q], hs[4 * q + 1], hs[4 * q + 2],
+                      hs[4 * q + 3], peer_xf);
+
+        int64_t slot0, g0;
+        int valid;
+        tg.blk.get(j, slot0, g0, valid);
+        if (valid < BN && t < BN && t >= valid) {
+          // a partial block: zero this CTA's latent rows past the last key so that masked
+          // keys contribute exact zeros to P.V whatever the ring holds there (the stage
+          // has landed: the score MMAs of this block have completed)
+          uint8_t* st = sm + OFF_KV + ((sw.gbase + jl) % NST) * BOX_BYTES + t * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4* p = reinterpret_cast<uint4*>(st + q * NST * BOX_BYTES);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) p[w] = make_uint4(0, 0, 0, 0);
+          }
+        }
+
+        // full scores: add the peer's partial
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + wg], kph, abort, a.err, 0x203,
+                                                 (t << 16) | j))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 x = my_x[q * TM];
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+            s[8 * q + 2 * e] += f.x;
+            s[8 * q + 2 * e + 1] += f.y;
+          }
+        }
+        named_bar(1 + wg, TM);            // the whole buffer is read: hand it back
+        if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);
+
+        // masked raw maximum (scores are scaled inside the exponent)
+        const int64_t lim64 = k_end_row - g0;
+        const int lim = lim64 < valid ? (lim64 < 0 ? 0 : (int)lim64) : valid;
+        if (lim < BN) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+        }
+        float rmax = s[0];
+#pragma unroll
+        for (int c = 1; c < 64; ++c) rmax = fmaxf(rmax, s[c]);
+        const float mb = rmax * c2;
+
+        // running maximum after the previous block (published by the other warpgroup)
+        const int ow = wg ^ 1, oseq = sw.nbase[ow] + ((jl - 1) >> 1);
+        float m_prev = -INFINITY;
+        if (jl > 0) {
+          if (!__all_sync(FULL, mbar_wait(&bar[B_M + ow], oseq & 1, abort, a.err, 0x204,
+                                          (t << 16) | j))) {
+            ok = false;
+            break;
+          }
+          m_prev = m_sh[ow * TM + t];
+        }
+        float m = m_prev, fac = 1.f;
+        if (jl == 0) {
+          m = mb;
+        } else if (mb > m_prev + 8.f) {
+          m = mb;
+          fac = ex2(m_prev - m);
+        }
+        m_sh[wg * TM + t] = m;
+        mbar_arrive(&bar[B_M + wg]);
+
+        const float msub = m == -INFINITY ? 0.f : m;
+        uint32_t pk[32];
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2(fmaf(s[2 * c], c2, -msub));
+          const float p1 = ex2(fmaf(s[2 * c + 1], c2, -msub));
+          sum += p0 + p1;
+          pk[c] = pack_bf16(p0, p1);
+        }
+        l = l * ex2(m_last - msub) + sum;
+        m_last = m;
+        // O is rescaled (warp-collective TMEM access) after PV of the previous block;
+        // the P buffer of this warpgroup is free once PV of its previous block is done
+        if (jl > 0 && __any_sync(FULL, fac != 1.f)) {
+          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ow], oseq & 1, abort, a.err, 0x205,
+                                          (t << 16) | j))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          rescale_row(tmem + lane_base + O_COL, fac);
+        }
         if (!__all_sync(FULL, mbar_wait(&bar[B_PE + wg], kph ^ 1, abort, a.err, 0x206,
                                         (t << 16) | j))) {
           ok = false;
           break;
         }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar[B_PF + wg]);
       }
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bar[B_PF + wg]);
-    }
+      if (!__all_sync(FULL, ok)) break;
 
-    // ------------------------------------------------------------ epilogue
-    if (ok) ok = mbar_wait(&bar[B_DONE], 0, abort, a.err, 0x401, t);
-    ok = __all_sync(FULL, ok);
-    tc_fence_after();
-    l_sh[(wg * 2) * TM + t] = l;
-    l_sh[(wg * 2 + 1) * TM + t] = m_last;
-    named_bar(3, 2 * TM);
-    const float l0 = l_sh[t], m0 = l_sh[TM + t], l1 = l_sh[2 * TM + t], m1 = l_sh[3 * TM + t];
-    const float mf = fmaxf(m0, m1);
-    const float lt = l0 * ex2(m0 - mf) + l1 * ex2(m1 - mf);
-    const float inv = lt > 0.f ? 1.f / lt : 0.f;
-    if (wg == 0 && rank == 0 && a.lse && row_valid && ok)
-      a.lse[grow] = (mf + log2f(lt)) * 0.69314718055994530942f;
-    bf16* dst = a.o_lat + grow * G.Dc + rank * HALF;
-#pragma unroll 1
-    for (int c = wg * (HALF / 2); c < (wg + 1) * (HALF / 2); c += 32) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_base + O_COL + c, v);
-      tmem_wait_ld();
-      if (ok && row_valid) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
-          w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
-          w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
-          w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
-          reinterpret_cast<uint4*>(dst + c)[q] = w;
+      // the next segment's Q may enter TMEM once this segment's score MMAs are done
+      const uint32_t kph = sw.k & 1;
+      {
+        SegWalk nx = sw;
+        nx.next(a);
+        if (nx.valid()) {
+          if (!__all_sync(FULL, mbar_wait(&bar[B_QKDONE], kph, abort, a.err, 0x301, t))) break;
+          tc_fence_after();
+          load_q(a, tmem + lane_base + Q_COL, nx.tg.grow0 + t, nx.tg.row0 + t < nx.tg.rows_b,
+                 rank, wg);
+          tc_fence_before();
+          mbar_arrive(&bar[B_QREADY]);
         }
       }
+
+      // ---------------------------------------------------------- segment epilogue
+      if (!__all_sync(FULL, mbar_wait(&bar[B_SEGDONE], kph, abort, a.err, 0x401, t))) break;
+      tc_fence_after();
+      l_sh[(wg * 2) * TM + t] = l;
+      l_sh[(wg * 2 + 1) * TM + t] = m_last;
+      named_bar(3, 2 * TM);
+      const float l0 = l_sh[t], m0 = l_sh[TM + t], l1 = l_sh[2 * TM + t], m1 = l_sh[3 * TM + t];
+      named_bar(3, 2 * TM);                  // both warpgroups have read (l, m)
+      const float mf = fmaxf(m0, m1);
+      const float lt = (m0 > -INFINITY ? l0 * ex2(m0 - mf) : 0.f) +
+                       (m1 > -INFINITY ? l1 * ex2(m1 - mf) : 0.f);
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float lse_v = lt > 0.f ? (mf + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+      const bool part = sw.partial();
+      if (wg == 0 && rank == 0 && row_valid) {
+        if (part)
+          a.ws_lse[(int64_t)sw.slot * TM + t] = lse_v;
+        else if (a.lse)
+          a.lse[grow] = lse_v;
+      }
+#pragma unroll 1
+      for (int c = wg * (HALF / 2); c < (wg + 1) * (HALF / 2); c += 32) {
+        uint32_t v[32];
+        if (n > 0) {
+          tmem_ld32(tmem + lane_base + O_COL + c, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = 0u;
+        }
+        if (!row_valid) continue;
+        if (part) {
+          float4* dst = reinterpret_cast<float4*>(a.ws_o + ((int64_t)sw.slot * TM + t) * G.Dc +
+                                                  rank * HALF + c);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv,
+                                 __uint_as_float(v[4 * q + 1]) * inv,
+                                 __uint_as_float(v[4 * q + 2]) * inv,
+                                 __uint_as_float(v[4 * q + 3]) * inv);
+        } else {
+          bf16* dst = a.o_lat + grow * G.Dc + rank * HALF + c;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+            w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+            w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+            w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+            reinterpret_cast<uint4*>(dst)[q] = w;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[B_OFREE]);
     }
   }
 
@@ -552,13 +688,93 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
 }
 
+// Split tiles to merge: tile[i] has the partial segments in workspace slots
+// [piece0[i], piece0[i + 1]).
+struct CombineList {
+  int32_t n;
+  int32_t tile[MAXC];
+  int32_t piece0[MAXC + 1];
+};
+
+// One CTA per (split tile, row), 4 latent dims per thread: the output is the partials
+// weighted by exp(lse_p - lse), lse = log sum_p exp(lse_p).
+__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ AttnArgs a,
+                                                      const __grid_constant__ CombineList cl) {
+  const int i = blockIdx.x / TM, r = blockIdx.x % TM;
+  const TileGeo tg =
+      tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, cl.tile[i]);
+  if (tg.row0 + r >= tg.rows_b) return;
+  const int64_t grow = tg.grow0 + r;
+  const int p0 = cl.piece0[i], p1 = cl.piece0[i + 1];
+  float mx = -INFINITY;
+  for (int p = p0; p < p1; ++p) mx = fmaxf(mx, a.ws_lse[(int64_t)p * TM + r]);
+  const int d = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  if (mx > -INFINITY) {
+    for (int p = p0; p < p1; ++p) {
+      const float lp = a.ws_lse[(int64_t)p * TM + r];
+      if (!(lp > -INFINITY)) continue;
+      const float w = expf(lp - mx);
+      wsum += w;
+      const float4 o =
+          *reinterpret_cast<const float4*>(a.ws_o + ((int64_t)p * TM + r) * a.g.Dc + d);
+      acc.x += w * o.x;
+      acc.y += w * o.y;
+      acc.z += w * o.z;
+      acc.w += w * o.w;
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint2 out;
+  out.x = pack_bf16(acc.x * inv, acc.y * inv);
+  out.y = pack_bf16(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(a.o_lat + grow * a.g.Dc + d) = out;
+  if (threadIdx.x == 0 && a.lse) a.lse[grow] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+}
+
+// Clusters of the attention kernel that can be resident at once on the current device
+// (one CTA per SM; a cluster needs two SMs of one GPC), capped at MAXC.  The first call
+// on a device also opts the kernel in to its shared memory.  0 on failure.
+int cluster_slots() {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  if (cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           ATT_SMEM) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * MAXC);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = ATT_SMEM;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attend_kernel, &cfg) != cudaSuccess || n < 1) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    n = sms / 2;
+  }
+  n = n < 1 ? 1 : (n > MAXC ? MAXC : n);
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc + 1) * sizeof(float); }
+
 }  // namespace
 
 bool tc_attend_supported(const Geo& g) { return g.Dc == 2 * HALF && g.Dr == 64; }
 
+size_t tc_attend_workspace(const Geo& g) { return 2 * (size_t)cluster_slots() * slot_bytes(g); }
+
+
 cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
                       const void* cache, int64_t k_first, int64_t n_keys, float scale,
-                      void* o_lat, float* lse, unsigned int* err, cudaStream_t st) {
+                      void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
+                      unsigned int* err, cudaStream_t st) {
   CUtensorMap K, KR, QR;
   {
     uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.S, (uint64_t)g.B};
@@ -574,13 +790,8 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     uint32_t b[2] = {32, TM};
     if (!make_tmap_bf16(&QR, q_abs, 2, d, s, b, true)) return cudaErrorInvalidValue;
   }
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const int ncl = cluster_slots();
+  if (ncl == 0) return cudaErrorInvalidDevice;
   AttnArgs a{};
   a.g = g;
   a.n_q = n_q; a.q_first = q_first; a.k_first = k_first; a.n_keys = n_keys;
@@ -590,11 +801,89 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.lse = lse;
   a.tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
   a.err = err;
-  const int64_t tiles = (int64_t)g.B * a.tiles_per_batch;
-  attend_kernel<<<(unsigned)(2 * tiles), NTHREADS, ATT_SMEM, st>>>(K, KR, QR, a);
+  const int T = g.B * a.tiles_per_batch;
+
+  // ---- schedule: the blocks of all tiles end to end, one equal range per cluster
+  const bool split = workspace != nullptr && workspace_bytes >= tc_attend_workspace(g);
+  std::vector<int64_t> pre(T + 1, 0);
+  std::vector<int> nbt(T);
+  for (int t = 0; t < T; ++t) {
+    nbt[t] = tile_geo(g, n_q, q_first, k_first, n_keys, a.tiles_per_batch, t).blk.nblk;
+    pre[t + 1] = pre[t] + nbt[t];
+  }
+  const int64_t W = pre[T];
+  Sched sc{};
+  int G;
+  if (split && W > 0) {
+    // cut c at block W*c/G; tiles without blocks go with the range before them
+    G = (int)(W < ncl ? W : ncl);
+    int t = 0;
+    for (int c = 1; c <= G; ++c) {
+      const int64_t pos = W * c / G;
+      while (t < T && pre[t + 1] <= pos) ++t;      // tile holding block `pos`
+      sc.cut_tile[c] = t;
+      sc.cut_blk[c] = t < T ? (int)(pos - pre[t]) : 0;
+    }
+  } else {
+    // cuts on tile boundaries: the first one at or past an equal share of the blocks
+    // (of the tiles when there are no blocks)
+    G = T < ncl ? T : ncl;
+    int t = 0;
+    for (int c = 1; c <= G; ++c) {
+      if (c == G) {
+        t = T;
+      } else if (W > 0) {
+        const int64_t pos = W * c / G;
+        while (t < T && pre[t] < pos) ++t;
+      } else {
+        t = (int)((int64_t)T * c / G);
+      }
+      sc.cut_tile[c] = t;
+      sc.cut_blk[c] = 0;
+    }
+  }
+  sc.cut_tile[0] = 0;
+  sc.cut_blk[0] = 0;
+  // partial segments: their workspace slots, and the tiles to combine
+  CombineList cl{};
+  int nslot = 0;
+  for (int c = 0; c < G; ++c) {
+    sc.slot0[c] = nslot;
+    int t = sc.cut_tile[c], jb = sc.cut_blk[c];
+    const int tend = sc.cut_tile[c + 1], bend = sc.cut_blk[c + 1];
+    while (t < tend || (t == tend && jb < bend)) {
+      const int je = t == tend ? bend : nbt[t];
+      if (jb > 0 || je < nbt[t]) {
+        if (cl.n == 0 || cl.tile[cl.n - 1] != t) {
+          if (cl.n == MAXC) return cudaErrorInvalidValue;   // at most G - 1 cuts split
+          cl.piece0[cl.n] = nslot;
+          cl.tile[cl.n++] = t;
+        }
+        ++nslot;
+      }
+      ++t;
+      jb = 0;
+    }
+  }
+  cl.piece0[cl.n] = nslot;
+  if (nslot > 2 * ncl) return cudaErrorInvalidValue;    // at most two per cluster
+  if (nslot > 0) {
+    a.ws_o = (float*)workspace;
+    a.ws_lse = a.ws_o + (size_t)2 * ncl * TM * g.Dc;
+  }
+  if (G == 0) return cudaSuccess;
+
+  attend_kernel<<<(unsigned)(2 * G), NTHREADS, ATT_SMEM, st>>>(K, KR, QR, a, sc);
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) count_launches(1);
-  return e;
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  if (cl.n > 0) {
+    combine_kernel<<<(unsigned)(cl.n * TM), 128, 0, st>>>(a, cl);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+  }
+  return cudaSuccess;
 }
 
 }  // namespace mla

@@ -201,3 +201,49 @@ def test_single_frame_window_and_last_query(cuda_ok):
                    wl.softmax_scale, o1, None, ws, ws_n)
     torch.cuda.synchronize()
     P.tol_check(P.download(o1)[:, 0], lat[:, last], wl.dtype, "o_lat one query")
+
+
+def _attend(r, wl, use_ws):
+    import latent_kv_cache_write_b200 as mla
+    T = wl.n_queries
+    o = torch.empty((wl.batch, T, wl.n_heads, wl.d_latent), dtype=torch.bfloat16, device=P.DEV)
+    lse = torch.empty((wl.batch, T, wl.n_heads), dtype=torch.float32, device=P.DEV)
+    ws, nws = None, 0
+    if use_ws:
+        nws = mla.mla_attend_workspace_size(r.shape, T, wl.n_keys)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=P.DEV)
+    mla.mla_attend(r.shape, r.q_abs, T, wl.q_first_tok, r.cache, wl.k_first_tok, wl.n_keys,
+                   wl.softmax_scale, o, lse, ws, nws)
+    torch.cuda.synchronize()
+    assert mla.mla_device_error() == 0
+    return P.download(o), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("use_ws", [True, False], ids=["split_keys", "whole_tiles"])
+def test_schedule_many_segments(cuda_ok, use_ws):
+    """136 tiles of 5 key blocks: more blocks than SM pairs, so every cluster walks
+    several segments (tile switches inside one launch); with a workspace the cuts also
+    split tiles (partials merged by the combine kernel), without one they fall on tile
+    boundaries.  All rows against the oracle."""
+    wl = C.small_variant(C.VIDEO_CHUNK).scaled(name="video_chunk_sched", batch=8,
+                                               n_heads=32, chunk_frames=1)
+    r = P.run_chunk(P.populate(wl, seed=5))
+    lat_ref, lse_ref = O.attend_latent(P.download(r.q_abs), P.download(r.cache), wl.q_first_tok,
+                                       wl.k_first_tok, wl.n_keys, wl.softmax_scale, wl)
+    o, lse = _attend(r, wl, use_ws)
+    P.tol_check(o, lat_ref, wl.dtype, "o_lat")
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=2e-2)
+
+
+def test_schedule_split_matches_whole(cuda_ok):
+    """The split-key and the whole-tile schedules give the same attention (up to the
+    rounding of the partial merge) on the full decode shape, where 64 tiles are fewer
+    than the SM pairs."""
+    wl = C.DECODE
+    r = P.populate(wl, seed=2)
+    r = P.run_chunk(r, with_lse=False)
+    o1, l1 = _attend(r, wl, True)
+    o2, l2 = _attend(r, wl, False)
+    err = float(np.linalg.norm(o1 - o2) / np.linalg.norm(o2))
+    assert err <= 4e-3, err
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-3)

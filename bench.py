@@ -195,24 +195,28 @@ class Step:
         self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.ws_bytes = mla.mla_attend_workspace_size(self.shape, T, wl.n_keys)
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
-        self.ev_attend = []
+    STAGES = ("cache_write", "absorb_q", "attend", "up_v")
 
-    def run(self, inp=None, attend_events=None):
+    def run(self, inp=None, ev=None):
+        """One step; with `ev` (5 CUDA events) the boundaries between its calls are
+        recorded on the current stream, the one the library launches on."""
         wl, mla = self.wl, self.mla
         inp = inp or self.dev_in
         T = wl.n_queries
         F = wl.tokens_per_frame
+        mark = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        mark(0)
         mla.mla_cache_write(self.shape, inp["h"], wl.d_model, T, wl.first_chunk_frame * F,
                             self.w["w_dkv"], self.w["w_kr"], self.cache)
+        mark(1)
         mla.mla_absorb_q(self.shape, inp["q_nope"], inp["q_rope"], T, wl.q_first_tok,
                          self.w["w_uk"], self.q_abs)
-        if attend_events is not None:
-            attend_events[0].record()
+        mark(2)
         mla.mla_attend(self.shape, self.q_abs, T, wl.q_first_tok, self.cache, wl.k_first_tok,
                        wl.n_keys, wl.softmax_scale, self.o_lat, self.lse, self.ws, self.ws_bytes)
-        if attend_events is not None:
-            attend_events[1].record()
+        mark(3)
         mla.mla_up_v(self.shape, self.o_lat, T, self.w["w_uv"], self.out)
+        mark(4)
 
     def run_e2e(self):
         """Host buffers in, host buffer out: copies inside the timed region."""
@@ -226,23 +230,23 @@ def torch_int16(torch):
     return torch.int16
 
 
-def time_steps(torch, fn, steps, flush, with_attend=False):
+def time_steps(torch, fn, steps, flush, n_marks=0):
     """Per step: flush L2 (untimed), then CUDA events around the step on the current
-    stream.  Returns (step ms list, attend ms list)."""
-    st, at = [], []
+    stream.  Returns (step ms list, per-interval ms lists between the n_marks events
+    the step records itself)."""
+    st, parts = [], [[] for _ in range(max(0, n_marks - 1))]
     for _ in range(steps):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) \
-            if with_attend else None
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(n_marks)] or None
         e0.record()
-        fn(a)
+        fn(marks)
         e1.record()
         torch.cuda.synchronize()
         st.append(e0.elapsed_time(e1))
-        if a:
-            at.append(a[0].elapsed_time(a[1]))
-    return st, at
+        for i in range(n_marks - 1):
+            parts[i].append(marks[i].elapsed_time(marks[i + 1]))
+    return st, parts
 
 
 def decode_leg(torch, mla, steps, warmup, flush):
@@ -349,8 +353,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        ms, attend_ms = time_steps(torch, lambda a: step.run(attend_events=a), args.steps, flush,
-                                   with_attend=True)
+        ms, parts = time_steps(torch, lambda ev: step.run(ev=ev), args.steps, flush, n_marks=5)
     torch.cuda.synchronize()
     launches = mla.mla_kernel_launches() - n0
     if world > 1:
@@ -375,7 +378,8 @@ def run_ours(args):
     ms_step = t_max / args.steps
     value = world * flops_step * args.steps / (t_max * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
-    att_ms = statistics.mean(attend_ms)
+    kernels_ms = {k: statistics.mean(v) for k, v in zip(Step.STAGES, parts)}
+    att_ms = kernels_ms["attend"]
     achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     dec = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush) if rank == 0 else None
@@ -409,7 +413,7 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "decode": dec,
             "clocks": clocks.summary(),
-            "kernels_ms": {"attend": att_ms},
+            "kernels_ms": kernels_ms,
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()

@@ -73,6 +73,20 @@ __device__ __forceinline__ int64_t rope_pos(const Geo& G, int64_t g, int p) {
   if (p < G.pairs[0] + G.pairs[1]) return y;
   return r - y * G.gw;
 }
+// The three axis positions (t, y, x) of token g, as doubles, computed once per token;
+// rope_axis_pos picks the one RoPE pair p turns by.
+struct RopeAxes {
+  double t, y, x;
+};
+__device__ __forceinline__ RopeAxes rope_axes(const Geo& G, int64_t g) {
+  const int64_t t = g / G.F;
+  const int64_t r = g - t * G.F;
+  const int64_t y = r / G.gw;
+  return RopeAxes{(double)t, (double)y, (double)(r - y * G.gw)};
+}
+__device__ __forceinline__ double rope_axis_pos(const Geo& G, const RopeAxes& ax, int p) {
+  return p < G.pairs[0] ? ax.t : (p < G.pairs[0] + G.pairs[1] ? ax.y : ax.x);
+}
 __device__ __forceinline__ double rope_inv_freq(const Geo& G, int p) {
   int j, n;
   if (p < G.pairs[0]) {
@@ -86,15 +100,16 @@ __device__ __forceinline__ double rope_inv_freq(const Geo& G, int p) {
 }
 
 // Rotate (a, b) by the angle pos * inv_freq: the product is formed in double, reduced
-// modulo 2*pi in double (Cody-Waite with a two-part 2*pi), then sin/cos are evaluated in
-// single precision; the error is ~1e-7 rad for any position the ABI admits.
+// modulo 2*pi in double (Cody-Waite with a two-part 2*pi) to [-pi, pi], where the
+// hardware sin/cos approximations (__sincosf) are accurate to ~4e-7 absolute; the
+// rotated pair is then rounded to bf16 (2^-9 relative).
 __device__ __forceinline__ void rope_rotate_fast(float& a, float& b, double pos, double inv_freq) {
   const double ang = pos * inv_freq;
   const double k = rint(ang * 0.15915494309189535);          // 1 / (2 pi)
   double r = fma(-k, 6.283185307179586, ang);                 // 2 pi, leading part
   r = fma(-k, 2.4492935982947064e-16, r);                     // 2 pi, trailing part
   float s, c;
-  sincosf((float)r, &s, &c);
+  __sincosf((float)r, &s, &c);
   const float na = a * c - b * s;
   const float nb = a * s + b * c;
   a = na;

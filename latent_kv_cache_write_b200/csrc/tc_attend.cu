@@ -19,8 +19,8 @@
 //
 // Two softmax warpgroups take alternate key blocks, so the exchange of one block
 // overlaps the exponentials of the other; they hand the running row maximum to each
-// other through shared memory.  An exchange buffer is handed back to the peer as soon as
-// its scores are read.  O is rescaled only when a row maximum grows by more than 8 (log2
+// other through shared memory.  The buffer the peer's partial scores land in takes P
+// once they are read.  O is rescaled only when a row maximum grows by more than 8 (log2
 // units).  Masking is frame-block-causal per row; a ring that wraps is walked as two
 // contiguous slot segments.
 //
@@ -51,56 +51,61 @@ using namespace tc;
 
 constexpr int TM = 128;                               // rows per tile
 constexpr int BN = 64;                                // keys per block
-constexpr int NST = 4;                                // K/V pipeline stages
 constexpr int HALF = 256;                             // latent dims per CTA
 constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
 constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB of latent per stage
 constexpr int RBOX_BYTES = BN * 32 * 2;               // 64 keys x 32 RoPE dims, 4 KB
 constexpr int STAGE_BYTES = LAT_BYTES + RBOX_BYTES;   // bytes one stage's loads bring
-// Shared-memory K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half,
-// 128-byte swizzle) of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage
-// s (64-byte swizzle) at OFF_KVR + s * RBOX_BYTES.  Consecutive stages are adjacent
-// within every box column, so one N=128 score MMA covers two consecutive 64-key blocks
-// unless their stages wrap around the ring.
 constexpr int QR_BYTES = TM * 32 * 2;                 // this CTA's Q RoPE part, 8 KB
-constexpr int X_BYTES = TM * BN * 2;                  // exchange buffer, 16 KB: the peer's
-                                                      // partial scores as fp16, chunk-major
-                                                      // [8 x 16 B][128 rows]
-constexpr int P_BYTES = TM * BN * 2;                  // P, bf16, 128-byte swizzled rows
+// Exchange buffer of a warpgroup, 16 KB: the peer's partial scores as fp16, chunk-major
+// [8 x 16 B][128 rows].  P buffer of a warpgroup, 16 KB: bf16, 128-byte swizzled rows.
+constexpr int XP_BYTES = TM * BN * 2;
 constexpr int NTHREADS = 352;
 constexpr int MAXC = 128;                             // clusters one launch can schedule
 
-constexpr int OFF_KV = 0;
-constexpr int OFF_KVR = OFF_KV + NST * LAT_BYTES;
-constexpr int OFF_QR = OFF_KVR + NST * RBOX_BYTES;
-constexpr int OFF_X = OFF_QR + QR_BYTES;              // [2] exchange buffers
-constexpr int OFF_P = OFF_X + 2 * X_BYTES;            // [2] P buffers
-constexpr int OFF_M = OFF_P + 2 * P_BYTES;            // running max handoff [2][128]
-constexpr int OFF_L = OFF_M + 2 * TM * 4;             // final (l, m) per warpgroup [2][2][128]
-constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
-
+// Shared-memory layout and barriers of the two pipeline depths.
+//   DEEP = false: 4 K/V stages; separate exchange and P buffers; an exchange buffer is
+//                 handed back to the peer as soon as its scores are read.
+//   DEEP = true:  5 K/V stages; P overwrites the exchange buffer once the scores are
+//                 read, and the PV product's commit, multicast to the peer, hands the
+//                 buffer back (the send of a block then waits for the peer's PV two
+//                 blocks earlier).  The deeper ring hides longer load latencies.
+// K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
+// swizzle) of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage s (64-byte
+// swizzle) at OFF_KVR + s * RBOX_BYTES.
 // A per-block barrier completes once per use of its buffer, a per-segment one once per
 // segment; a waiter counts the uses and waits on the parity of the count.
-enum {
-  B_KVF = 0,                // K/V stage loaded (TMA)
-  B_KVE = B_KVF + NST,      // K/V stage free (MMA commit after PV)
-  B_QR = B_KVE + NST,       // Q RoPE tile of a segment loaded (TMA)
-  B_QREADY,                 // Q latent half of a segment in TMEM (256 threads)
-  B_QKDONE,                 // every score MMA of a segment finished (MMA commit)
-  B_SEGDONE,                // every PV MMA of a segment finished (MMA commit)
-  B_OFREE,                  // O of a segment read out of TMEM (256 threads)
-  B_SF,                     // S buffer full (MMA commit)                  [2]
-  B_SE = B_SF + 2,          // S buffer read (128 threads)                 [2]
-  B_XF = B_SE + 2,          // peer's partial scores landed (tx bytes)     [2]
-  B_XE = B_XF + 2,          // peer read the scores sent it (1 remote)    [2]
-  B_PF = B_XE + 2,          // P complete, O rescaled (128)                [2]
-  B_PE = B_PF + 2,          // PV done (MMA commit)                        [2]
-  B_M = B_PE + 2,           // running max of a block published (128)      [2]
-  NBAR = B_M + 2
+template <bool DEEP>
+struct Lay {
+  static constexpr int NST = DEEP ? 5 : 4;
+  static constexpr bool MERGED = DEEP;
+  static constexpr int OFF_KV = 0;
+  static constexpr int OFF_KVR = OFF_KV + NST * LAT_BYTES;
+  static constexpr int OFF_QR = OFF_KVR + NST * RBOX_BYTES;
+  static constexpr int OFF_X = OFF_QR + QR_BYTES;                 // [2] exchange buffers
+  static constexpr int OFF_P = MERGED ? OFF_X : OFF_X + 2 * XP_BYTES;   // [2] P buffers
+  static constexpr int OFF_M = OFF_P + 2 * XP_BYTES;              // running max [2][128]
+  static constexpr int OFF_L = OFF_M + 2 * TM * 4;                // final (l, m) [2][2][128]
+  static constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
+  static constexpr int B_KVF = 0;               // K/V stage loaded (TMA)                [NST]
+  static constexpr int B_KVE = B_KVF + NST;     // K/V stage free (MMA commit after PV) [NST]
+  static constexpr int B_QR = B_KVE + NST;      // Q RoPE tile of a segment loaded (TMA)
+  static constexpr int B_QREADY = B_QR + 1;     // Q latent half of a segment in TMEM (256)
+  static constexpr int B_QKDONE = B_QR + 2;     // every score MMA of a segment finished
+  static constexpr int B_SEGDONE = B_QR + 3;    // every PV MMA of a segment finished
+  static constexpr int B_OFREE = B_QR + 4;      // O of a segment read out of TMEM (256)
+  static constexpr int B_SF = B_QR + 5;         // S buffer full (MMA commit)            [2]
+  static constexpr int B_SE = B_SF + 2;         // S buffer read (128)                   [2]
+  static constexpr int B_XF = B_SE + 2;         // peer's partial scores landed (tx)     [2]
+  static constexpr int B_XE = B_XF + 2;         // exchange buffer in the peer free       [2]
+  static constexpr int B_PF = B_XE + 2;         // P complete, O rescaled (128)          [2]
+  static constexpr int B_PE = B_PF + 2;         // PV done (MMA commit)                  [2]
+  static constexpr int B_M = B_PE + 2;          // running max of a block published (128) [2]
+  static constexpr int NBAR = B_M + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
 };
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int ATT_SMEM = OFF_MISC + 16 + 1024;
-static_assert(ATT_SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
 
 constexpr uint32_t O_COL = 0, Q_COL = 256, S_COL = 384;
 constexpr unsigned FULL = 0xffffffffu;
@@ -211,6 +216,8 @@ struct SegWalk {
     je = tile == tend ? bend : tg.blk.nblk;
   }
   __device__ int nb() const { return je - jb; }
+  // blocks of earlier segments taken by warpgroup w (a select, not an indexed load)
+  __device__ int done_by(int w) const { return w ? nbase[1] : nbase[0]; }
   __device__ bool partial() const { return jb > 0 || je < tg.blk.nblk; }
   __device__ void next(const AttnArgs& a) {
     const int n = nb();
@@ -257,16 +264,25 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, uint32_t tq, int64_t g
   tmem_wait_st();
 }
 
+template <bool DEEP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
                   const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ AttnArgs a,
                   const __grid_constant__ Sched sc) {
+  using LY = Lay<DEEP>;
+  constexpr int NST = LY::NST;
+  constexpr int OFF_KV = LY::OFF_KV, OFF_KVR = LY::OFF_KVR, OFF_QR = LY::OFF_QR;
+  constexpr int OFF_X = LY::OFF_X, OFF_P = LY::OFF_P, OFF_M = LY::OFF_M, OFF_L = LY::OFF_L;
+  constexpr int B_KVF = LY::B_KVF, B_KVE = LY::B_KVE, B_QR = LY::B_QR, B_QREADY = LY::B_QREADY;
+  constexpr int B_QKDONE = LY::B_QKDONE, B_SEGDONE = LY::B_SEGDONE, B_OFREE = LY::B_OFREE;
+  constexpr int B_SF = LY::B_SF, B_SE = LY::B_SE, B_XF = LY::B_XF, B_XE = LY::B_XE;
+  constexpr int B_PF = LY::B_PF, B_PE = LY::B_PE, B_M = LY::B_M;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + LY::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + LY::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(sm + LY::OFF_MISC + 4);
 
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -373,7 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int jl = 0; jl < n; ++jl) {
           const int w = jl & 1;                          // S buffer = warpgroup
           const int g = sw.gbase + jl, s = g % NST;
-          const int q = sw.nbase[w] + (jl >> 1);         // S buffer use
+          const int q = sw.done_by(w) + (jl >> 1);         // S buffer use
           ok = mbar_wait(&bar[B_KVF + s], (g / NST) & 1, abort, a.err, 0x105, g);
           if (ok) ok = mbar_wait(&bar[B_SE + w], (q & 1) ^ 1, abort, a.err, 0x106, g);
           if (!ok) break;
@@ -387,7 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   } else if (warp == 10) {
     // ------------------------------------------------------------ PV issuer
     // O += P . V in block order as each P is ready; the commits free the K/V stage for
-    // the next load and the P buffer, and let the softmax rescale O.  A segment starts
+    // the next load and the P buffer, let the softmax rescale O, and with merged
+    // exchange/P buffers (multicast to the peer) let the peer send its next partial
+    // scores into the buffer that held P.  A segment starts
     // once the previous segment's O has been read out (its first PV overwrites O); its
     // last commit also covers its score MMAs: a block's P exists only after its scores
     // were read.
@@ -398,13 +416,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (sw.k > 0) ok = mbar_wait(&bar[B_OFREE], (sw.k - 1) & 1, abort, a.err, 0x108, sw.k);
         const int n = sw.nb();
         for (int jl = 0; ok && jl < n; ++jl) {
-          const int pb = jl & 1, seq = sw.nbase[pb] + (jl >> 1);
+          const int pb = jl & 1, seq = sw.done_by(pb) + (jl >> 1);
           const int g = sw.gbase + jl, s = g % NST;
           ok = mbar_wait(&bar[B_PF + pb], seq & 1, abort, a.err, 0x104, g);
           if (!ok) break;
           tc_fence_after();
           const uint32_t v0 = smem_u32(sm + OFF_KV + s * BOX_BYTES);
-          const uint32_t pa = smem_u32(sm + OFF_P + pb * P_BYTES);
+          const uint32_t pa = smem_u32(sm + OFF_P + pb * XP_BYTES);
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks)
             mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
@@ -412,6 +430,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                    (jl > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar[B_PE + pb]);
           mma_commit(&bar[B_KVE + s]);
+          if constexpr (LY::MERGED) mma_commit_cluster(&bar[B_XE + pb], (uint16_t)(1u << peer));
         }
         if (ok) mma_commit(&bar[B_SEGDONE]);
       }
@@ -423,11 +442,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     float* m_sh = reinterpret_cast<float*>(sm + OFF_M);
     float* l_sh = reinterpret_cast<float*>(sm + OFF_L);
-    const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * X_BYTES), peer) + (uint32_t)t * 16;
+    const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * XP_BYTES), peer) + (uint32_t)t * 16;
     const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
-    const uint4* my_x = reinterpret_cast<const uint4*>(sm + OFF_X + wg * X_BYTES) + t;
-    uint8_t* prow = sm + OFF_P + wg * P_BYTES + t * 128;     // P row t
     const uint32_t peer_xe = mapa(smem_u32(&bar[B_XE + wg]), peer);
+    const uint4* my_x = reinterpret_cast<const uint4*>(sm + OFF_X + wg * XP_BYTES) + t;
+    uint8_t* prow = sm + OFF_P + wg * XP_BYTES + t * 128;    // P row t
     const float c2 = a.scale_log2;
     bool ok = true;
 
@@ -448,11 +467,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       float m_last = -INFINITY, l = 0.f;       // this warpgroup's running sum and its max
       for (int jl = wg; jl < n; jl += 2) {
         const int j = sw.jb + jl;              // block of the tile
-        const int seq = sw.nbase[wg] + (jl >> 1);
+        const int seq = sw.done_by(wg) + (jl >> 1);
         const uint32_t kph = seq & 1;
-        // arm this block's exchange: the peer's asynchronous stores complete X_BYTES of
+        // arm this block's exchange: the peer's asynchronous stores complete XP_BYTES of
         // transactions on it (they may land before or after this arrive)
-        if (t == 0) mbar_expect_tx(&bar[B_XF + wg], X_BYTES);
+        if (t == 0) mbar_expect_tx(&bar[B_XF + wg], XP_BYTES);
         if (!__all_sync(FULL, mbar_wait(&bar[B_SF + wg], kph, abort, a.err, 0x201, (t << 16) | j))) {
           ok = false;
           break;
@@ -460,21 +479,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         float s[64];
         {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + S_COL + wg * BN, v);
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_base + S_COL + wg * BN, v0);
+          tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v1);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(v[c]);
-          tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(v[c]);
+          for (int c = 0; c < 32; ++c) {
+            s[c] = __uint_as_float(v0[c]);
+            s[32 + c] = __uint_as_float(v1[c]);
+          }
         }
         tc_fence_before();
         mbar_arrive(&bar[B_SE + wg]);
 
-        // send this CTA's partial scores into the peer's buffer once the peer has read
-        // what was sent two blocks ago
+        // send this CTA's partial scores into the peer's buffer once the peer is done
+        // with it: it has read what was sent two blocks ago (and, with merged buffers,
+        // its PV has read the P held there)
         if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], kph ^ 1, abort, a.err, 0x202,
                                                  (t << 16) | j))) {
           ok = false;
@@ -529,8 +549,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             s[8 * q + 2 * e + 1] += f.y;
           }
         }
-        named_bar(1 + wg, TM);            // the whole buffer is read: hand it back
-        if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);
+        named_bar(1 + wg, TM);            // the whole buffer is read
+        if constexpr (!LY::MERGED) {
+          if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);   // hand it back
+        }
 
         // masked raw maximum (scores are scaled inside the exponent)
         const int64_t lim64 = k_end_row - g0;
@@ -545,7 +567,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const float mb = rmax * c2;
 
         // running maximum after the previous block (published by the other warpgroup)
-        const int ow = wg ^ 1, oseq = sw.nbase[ow] + ((jl - 1) >> 1);
+        const int ow = wg ^ 1, oseq = sw.done_by(ow) + ((jl - 1) >> 1);
         float m_prev = -INFINITY;
         if (jl > 0) {
           if (!__all_sync(FULL, mbar_wait(&bar[B_M + ow], oseq & 1, abort, a.err, 0x204,
@@ -577,8 +599,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         l = l * ex2(m_last - msub) + sum;
         m_last = m;
-        // O is rescaled (warp-collective TMEM access) after PV of the previous block;
-        // the P buffer of this warpgroup is free once PV of its previous block is done
+        // O is rescaled (warp-collective TMEM access) after PV of the previous block.
+        // The P buffer is free once PV of this warpgroup's previous block has read it
+        // (with merged buffers that is implied: the peer sent this block's scores into
+        // it only then).
         if (jl > 0 && __any_sync(FULL, fac != 1.f)) {
           if (!__all_sync(FULL, mbar_wait(&bar[B_PE + ow], oseq & 1, abort, a.err, 0x205,
                                           (t << 16) | j))) {
@@ -588,10 +612,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           tc_fence_after();
           rescale_row(tmem + lane_base + O_COL, fac);
         }
-        if (!__all_sync(FULL, mbar_wait(&bar[B_PE + wg], kph ^ 1, abort, a.err, 0x206,
-                                        (t << 16) | j))) {
-          ok = false;
-          break;
+        if constexpr (!LY::MERGED) {
+          if (!__all_sync(FULL, mbar_wait(&bar[B_PE + wg], kph ^ 1, abort, a.err, 0x206,
+                                          (t << 16) | j))) {
+            ok = false;
+            break;
+          }
         }
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -674,6 +700,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       tc_fence_before();
       mbar_arrive(&bar[B_OFREE]);
     }
+    // with merged buffers the peer's last PV commit arrives on this CTA's barrier: let it
+    // land before exit
+    if constexpr (LY::MERGED) {
+      if (ok && !sw.valid() && sw.done_by(wg) > 0)
+        mbar_wait_cluster(&bar[B_XE + wg], (sw.done_by(wg) - 1) & 1, abort, a.err, 0x402, t);
+    }
   }
 
   // ------------------------------------------------------------ teardown
@@ -743,15 +775,21 @@ int cluster_slots() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (dev < 64 && cached[dev] > 0) return cached[dev];
-  if (cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           ATT_SMEM) != cudaSuccess)
+  if (cudaFuncSetAttribute(attend_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Lay<false>::SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(attend_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Lay<true>::SMEM) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * MAXC);
   cfg.blockDim = dim3(NTHREADS);
-  cfg.dynamicSmemBytes = ATT_SMEM;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, attend_kernel, &cfg) != cudaSuccess || n < 1) {
+  int n = 0, n2 = 0;
+  cfg.dynamicSmemBytes = Lay<false>::SMEM;
+  cudaError_t e1 = cudaOccupancyMaxActiveClusters(&n, attend_kernel<false>, &cfg);
+  cfg.dynamicSmemBytes = Lay<true>::SMEM;
+  cudaError_t e2 = cudaOccupancyMaxActiveClusters(&n2, attend_kernel<true>, &cfg);
+  if (e1 == cudaSuccess && e2 == cudaSuccess) n = n < n2 ? n : n2;
+  if (e1 != cudaSuccess || e2 != cudaSuccess || n < 1) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return 0;
@@ -873,7 +911,14 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   }
   if (G == 0) return cudaSuccess;
 
-  attend_kernel<<<(unsigned)(2 * G), NTHREADS, ATT_SMEM, st>>>(K, KR, QR, a, sc);
+  // A tile whose keys no other tile reads streams them from HBM: the deeper ring hides
+  // that latency.  Keys shared by many tiles mostly hit in L2, where the shorter
+  // hand-back of the exchange buffer matters more (both measured on the video-chunk
+  // and decode shapes).
+  if (a.tiles_per_batch <= 2)
+    attend_kernel<true><<<(unsigned)(2 * G), NTHREADS, Lay<true>::SMEM, st>>>(K, KR, QR, a, sc);
+  else
+    attend_kernel<false><<<(unsigned)(2 * G), NTHREADS, Lay<false>::SMEM, st>>>(K, KR, QR, a, sc);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);

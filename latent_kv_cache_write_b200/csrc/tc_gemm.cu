@@ -23,7 +23,10 @@ constexpr int A_BYTES = GBM * GBK * 2;           // 16 KB
 constexpr int B_BYTES = GBN * GBK * 2;           // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int MAX_PAIRS = 512;                   // RoPE pairs with a table entry (d_R <= 1024)
-constexpr int GEMM_SMEM = GSTAGES * STAGE_BYTES + 1024 + 256 + MAX_PAIRS * 8;
+constexpr int STG_BYTES = 32 * 64;                // per epilogue warp: 32 rows x 32 cols bf16
+constexpr int OFF_TAB = GSTAGES * STAGE_BYTES + 256;
+constexpr int OFF_STG = OFF_TAB + MAX_PAIRS * 8;
+constexpr int GEMM_SMEM = OFF_STG + 4 * STG_BYTES + 1024;
 
 enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
 
@@ -53,7 +56,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   uint64_t* acce = accf + 2;                     // accumulator drained [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  double* inv_freq = reinterpret_cast<double*>(smem + GSTAGES * STAGE_BYTES + 256);
+  double* inv_freq = reinterpret_cast<double*>(smem + OFF_TAB);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nm = (p.M + GBM - 1) / GBM, nn = (p.N + GBN - 1) / GBN;
@@ -153,9 +156,15 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue warps
+    // Thread r drains TMEM row r of its warp's lane quarter 32 columns at a time, into a
+    // per-warp staging buffer (2 KB, 16-byte chunks XOR-swizzled by row so that neither
+    // the row-wise writes nor the chunk-wise reads conflict); the warp then writes the
+    // 32 rows as 64-byte segments, four lanes per row, instead of one scattered row per
+    // lane.
     const int r = (warp & 3) * 32 + lane;       // TMEM lane quarter = warp id % 4
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const Geo& G = p.geo;
+    uint8_t* stg = smem + OFF_STG + (warp - 2) * STG_BYTES;
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
       int m0, n0, z;
@@ -165,6 +174,20 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                                                          0x13, (r << 16) | tc));
       tc_fence_after();
       const int64_t m = m0 + r;
+      const bool row_ok = m < p.M;
+      // this row's output base (element offset of column 0) and, for the cache, its token
+      int64_t base = 0, g = 0;
+      RopeAxes ax{0.0, 0.0, 0.0};
+      if (p.mode == MODE_CACHE) {
+        const int64_t b = m / p.rows_per_batch;
+        g = p.first_tok + (m - b * p.rows_per_batch);
+        base = (b * G.S + g % G.S) * G.row;
+        if (row_ok && G.Dr > 0) ax = rope_axes(G, g);
+      } else if (p.mode == MODE_ABSORB) {
+        base = (m * G.H + z) * G.row;
+      } else {
+        base = (m * G.H + z) * G.Dn;
+      }
       const uint32_t trow = tmem + lane_base + acc * GBN;
       for (int c0 = 0; c0 < GBN; c0 += 32) {
         uint32_t v[32];
@@ -174,55 +197,41 @@ __global__ void __launch_bounds__(GTHREADS, 1)
           tc_fence_before();
           mbar_arrive(&acce[acc]);              // accumulator may be overwritten
         }
-        if (!ok || m >= p.M) continue;
-        const int n = n0 + c0;                  // output column of v[0]
-        if (n >= p.N) continue;
+        const int n = n0 + c0;                  // output column of v[0] (warp-uniform)
+        if (!ok || n >= p.N) continue;
         float f[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-        bf16* dst;
-        if (p.mode == MODE_CACHE) {
-          const int64_t b = m / p.rows_per_batch;
-          const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
-          const int64_t slot = g % G.S;
-          if (n >= p.n_split) {
-#pragma unroll 4
-            for (int j = 0; j < 32; j += 2) {
-              const int q = (n + j - p.n_split) / 2;
-              rope_rotate_fast(f[j], f[j + 1], (double)rope_pos(G, g, q), inv_freq[q]);
-            }
-          }
-          dst = p.out + (b * G.S + slot) * G.row + n;
-        } else if (p.mode == MODE_ABSORB) {
-          dst = p.out + (m * G.H + z) * G.row + n;
-        } else {
-          dst = p.out + (m * G.H + z) * G.Dn + n;
-        }
-        const int valid = p.N - n < 32 ? p.N - n : 32;
-        if (valid == 32) {
+        if (p.mode == MODE_CACHE && n >= p.n_split && row_ok) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 w;
-            w.x = pack_bf16(f[8 * q + 0], f[8 * q + 1]);
-            w.y = pack_bf16(f[8 * q + 2], f[8 * q + 3]);
-            w.z = pack_bf16(f[8 * q + 4], f[8 * q + 5]);
-            w.w = pack_bf16(f[8 * q + 6], f[8 * q + 7]);
-            reinterpret_cast<uint4*>(dst)[q] = w;
+          for (int j = 0; j < 32; j += 2) {
+            const int q = (n + j - p.n_split) / 2;
+            rope_rotate_fast(f[j], f[j + 1], rope_axis_pos(G, ax, q), inv_freq[q]);
           }
-        } else {
-          for (int j = 0; j < valid; ++j) dst[j] = __float2bfloat16_rn(f[j]);
         }
+        uint4* srow = reinterpret_cast<uint4*>(stg + lane * 64);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          srow[q ^ ((lane >> 1) & 3)] =
+              make_uint4(pack_bf16(f[8 * q + 0], f[8 * q + 1]), pack_bf16(f[8 * q + 2], f[8 * q + 3]),
+                         pack_bf16(f[8 * q + 4], f[8 * q + 5]), pack_bf16(f[8 * q + 6], f[8 * q + 7]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = 8 * i + (lane >> 2), j = lane & 3;      // row of the warp, chunk
+          const int64_t rbase = __shfl_sync(0xffffffffu, base, rr);
+          if (m0 + (warp & 3) * 32 + rr < p.M) {
+            const uint4 w = reinterpret_cast<const uint4*>(stg + rr * 64)[j ^ ((rr >> 1) & 3)];
+            *reinterpret_cast<uint4*>(p.out + rbase + n + 8 * j) = w;
+          }
+        }
+        __syncwarp();
       }
-      if (ok && m < p.M && n0 == 0) {
-        if (p.mode == MODE_CACHE && p.slots) {
-          const int64_t b = m / p.rows_per_batch;
-          const int64_t g = p.first_tok + (m - b * p.rows_per_batch);
-          p.slots[m] = (int32_t)(g % G.S);
-        }
+      if (ok && row_ok && n0 == 0) {
+        if (p.mode == MODE_CACHE && p.slots) p.slots[m] = (int32_t)(g % G.S);
         if (p.mode == MODE_ABSORB && G.Dr > 0) {
           // q_abs[.., Dc:] = RoPE(q_R) for this tile's rows and head
-          const int64_t i = m % p.rows_per_batch;
-          const int64_t g = p.first_tok + i;
+          const RopeAxes qa = rope_axes(G, p.first_tok + m % p.rows_per_batch);
           const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + (m * G.H + z) * G.Dr);
           uint4* dst = reinterpret_cast<uint4*>(p.out + (m * G.H + z) * G.row + G.Dc);
           // 8 bf16 (4 pairs) per 16-byte vector; the loads of a chunk are issued together
@@ -239,7 +248,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 const int q = (c + u) * 4 + e;
                 const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
                 float a = f.x, b = f.y;
-                rope_rotate_fast(a, b, (double)rope_pos(G, g, q), inv_freq[q]);
+                rope_rotate_fast(a, b, rope_axis_pos(G, qa, q), inv_freq[q]);
                 w[e] = pack_bf16(a, b);
               }
               dst[c + u] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -294,6 +303,7 @@ cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap
 }  // namespace
 
 bool tc_gemm_supported(const Geo& g, int d_model) {
+  // every output width is a multiple of the epilogue's 32-column chunks
   return g.Dc % GBN == 0 && g.Dr % 64 == 0 && g.Dn % 64 == 0 && g.Dr / 2 <= MAX_PAIRS &&
          (d_model <= 0 || d_model % 64 == 0);
 }

@@ -160,6 +160,38 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * MLA_FIXED_SCRATCH_BYTES, mla_attend_fixed_scratch — mla_attend without a caller
+ * workspace.  The pages have no counterpart: this is an interface matter, not part of
+ * the method.
+ *
+ * For callers that cannot hand mla_attend a device workspace: a plain C host that
+ * holds only the tensors it was given and no device allocator of its own, or a serving
+ * loop that must not allocate between steps (cudaMalloc and cudaFree synchronise the
+ * device).  Instead of the workspace, the split-key partials (float32 partial outputs
+ * and log-sum-exps) go to one static device array of MLA_FIXED_SCRATCH_BYTES inside the
+ * library, 40 MiB per device (two partial slots of 128 x (d_latent + 1) floats for each
+ * resident pair of SMs: 37 MiB on a 148-SM B200).  The call allocates nothing.
+ *
+ * Arguments, results and errors are those of mla_attend (without workspace and
+ * workspace_bytes); the results equal mla_attend's with a full workspace.  In addition:
+ *   - MLA_ERR_UNSUPPORTED if this shape on the current device would need more scratch
+ *     than MLA_FIXED_SCRATCH_BYTES (mla_attend_workspace_size() > it);
+ *   - MLA_ERR_CUDA if the array's device address cannot be obtained.
+ * The first call on a device looks the array's address up (cudaGetSymbolAddress, with
+ * that device current) and should come before any stream capture.
+ * All calls on a device share the one array: calls that overlap in time (on different
+ * streams, or from different host threads without ordering) race on it and corrupt each
+ * other's results; calls ordered on one stream do not.  Nothing in the array needs to
+ * start at zero: every slot a call reads was written earlier in the same call.
+ */
+#define MLA_FIXED_SCRATCH_BYTES (40u * 1024u * 1024u)
+
+mla_status mla_attend_fixed_scratch(const mla_shape* shape, const void* q_abs, int64_t n_q,
+                                    int64_t q_first_tok, const void* cache,
+                                    int64_t k_first_tok, int64_t n_keys, float softmax_scale,
+                                    void* o_lat, float* lse, void* stream);
+
+/*
  * mla_up_v — step 5: per-head W_UV up-projection of the latent attention output
  * (concept page, "Low-rank joint compression": W^UV is applied on the output side).
  *   out[b][i][h] = w_uv[h] . o_lat[b][i][h]     ([d_nope, d_latent] x [d_latent])

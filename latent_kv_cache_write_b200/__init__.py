@@ -15,6 +15,7 @@ from . import native
 from .native import MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
+           "mla_attend_fixed_scratch",
            "mla_up_v", "mla_device_error", "mla_kernel_launches", "mla_device_error_info", "make_shape", "MlaShape", "MlaError"]
 
 
@@ -63,6 +64,14 @@ def mla_attend(shape: MlaShape, q_abs, n_q: int, q_first_tok: int, cache, k_firs
         ctypes.byref(shape), _ptr(q_abs), n_q, q_first_tok, _ptr(cache), k_first_tok, n_keys,
         softmax_scale, _ptr(o_lat), _ptr(lse), _ptr(workspace), workspace_bytes,
         _stream(stream)))
+
+
+def mla_attend_fixed_scratch(shape: MlaShape, q_abs, n_q: int, q_first_tok: int, cache,
+                             k_first_tok: int, n_keys: int, softmax_scale: float, o_lat,
+                             lse=None, stream=None) -> None:
+    native.check("mla_attend_fixed_scratch", native.lib().mla_attend_fixed_scratch(
+        ctypes.byref(shape), _ptr(q_abs), n_q, q_first_tok, _ptr(cache), k_first_tok, n_keys,
+        softmax_scale, _ptr(o_lat), _ptr(lse), _stream(stream)))
 
 
 def mla_up_v(shape: MlaShape, o_lat, n_q: int, w_uv, out, stream=None) -> None:

@@ -46,6 +46,9 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
                       void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
                       unsigned int* err, cudaStream_t st);
 
+// Address of the static split-key scratch (MLA_FIXED_SCRATCH_BYTES) on the current device.
+cudaError_t fixed_scratch(void** ptr);
+
 // Device address of the library's error word on the current device (nullptr on failure).
 unsigned int* device_error_word();
 

@@ -168,6 +168,27 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
                                  softmax_scale, o_lat, lse, (cudaStream_t)stream));
 }
 
+mla_status mla_attend_fixed_scratch(const mla_shape* shape, const void* q_abs, int64_t n_q,
+                                    int64_t q_first_tok, const void* cache,
+                                    int64_t k_first_tok, int64_t n_keys, float softmax_scale,
+                                    void* o_lat, float* lse, void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  // the static array replaces the caller's workspace; a shape and device that would
+  // need more is refused rather than run with a smaller schedule
+  const size_t need = mla_attend_workspace_size(shape, n_q, n_keys);
+  if (need > MLA_FIXED_SCRATCH_BYTES) return MLA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  size_t bytes = 0;
+  if (need > 0) {
+    if (fixed_scratch(&scratch) != cudaSuccess) return MLA_ERR_CUDA;
+    bytes = MLA_FIXED_SCRATCH_BYTES;
+  }
+  return mla_attend(shape, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys, softmax_scale,
+                    o_lat, lse, scratch, bytes, stream);
+}
+
 mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, const void* w_uv,
                     void* out, void* stream) {
   Geo g;

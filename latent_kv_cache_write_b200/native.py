@@ -37,6 +37,8 @@ SIGNATURES = {
     "mla_absorb_q": (_i32, [_P, _vp, _vp, _i64, _i64, _vp, _vp, _vp]),
     "mla_attend_workspace_size": (_sz, [_P, _i64, _i64]),
     "mla_attend": (_i32, [_P, _vp, _i64, _i64, _vp, _i64, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "mla_attend_fixed_scratch": (_i32, [_P, _vp, _i64, _i64, _vp, _i64, _i64, _f32, _vp, _vp,
+                                        _vp]),
     "mla_up_v": (_i32, [_P, _vp, _i64, _vp, _vp, _vp]),
     "mla_status_string": (ctypes.c_char_p, [_i32]),
     "mla_device_error": (_i32, [_vp]),

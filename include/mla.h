@@ -169,7 +169,7 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
  * loop that must not allocate between steps (cudaMalloc and cudaFree synchronise the
  * device).  Instead of the workspace, the split-key partials (float32 partial outputs
  * and log-sum-exps) go to one static device array of MLA_FIXED_SCRATCH_BYTES inside the
- * library, 40 MiB per device (two partial slots of 128 x (d_latent + 1) floats for each
+ * library, 40 MiB per device (two partial slots of 128 x (d_latent + 2) floats for each
  * resident pair of SMs: 37 MiB on a 148-SM B200).  The call allocates nothing.
  *
  * Arguments, results and errors are those of mla_attend (without workspace and

@@ -13,8 +13,9 @@
 //     resident in TMEM as the A operand, the RoPE part from shared memory),
 //   - swaps partial scores (rounded to fp16) with its peer through distributed shared
 //     memory, so both CTAs hold the full scores of all 128 rows,
-//   - runs the online softmax of all 128 rows itself (both CTAs take bit-identical
-//     decisions: each adds the same two fp16-rounded partials),
+//   - runs the online softmax of all 128 rows itself (its own fp32 partial plus the
+//     peer's fp16-rounded one; the CTAs' row sums may differ in the last bits, and each
+//     normalises its own half of O with its own sum),
 //   - accumulates O_c += P . V_c (M=128, N=256) into its TMEM.
 //
 // Two softmax warpgroups take alternate key blocks, so the exchange of one block
@@ -118,7 +119,7 @@ struct AttnArgs {
   bf16* o_lat;
   float* lse;
   float* ws_o;              // partial outputs [slot][TM][Dc], fp32, normalised by their l
-  float* ws_lse;            // their natural log-sum-exps [slot][TM]
+  float* ws_lse;            // their natural log-sum-exps, one per CTA half [slot][2][TM]
   int tiles_per_batch;
   unsigned int* err;
 };
@@ -500,16 +501,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        // both CTAs add the same two fp16-rounded partials, so their softmax agrees bit
-        // for bit; the rounding is ~2^-11 of a partial score
+        // the peer receives this partial rounded to fp16 (~2^-11 of a partial score)
         uint32_t hs[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           __half2 h2 = __floats2half2_rn(s[2 * c], s[2 * c + 1]);
           hs[c] = *reinterpret_cast<uint32_t*>(&h2);
-          const float2 back = __half22float2(h2);
-          s[2 * c] = back.x;
-          s[2 * c + 1] = back.y;
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q)
@@ -658,10 +655,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const float lse_v = lt > 0.f ? (mf + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
       const bool part = sw.partial();
-      if (wg == 0 && rank == 0 && row_valid) {
+      if (wg == 0 && row_valid) {
         if (part)
-          a.ws_lse[(int64_t)sw.slot * TM + t] = lse_v;
-        else if (a.lse)
+          a.ws_lse[((int64_t)sw.slot * 2 + rank) * TM + t] = lse_v;
+        else if (a.lse && rank == 0)
           a.lse[grow] = lse_v;
       }
 #pragma unroll 1
@@ -729,7 +726,8 @@ struct CombineList {
 };
 
 // One CTA per (split tile, row), 4 latent dims per thread: the output is the partials
-// weighted by exp(lse_p - lse), lse = log sum_p exp(lse_p).
+// weighted by exp(lse_p - lse), lse = log sum_p exp(lse_p), each half of the dims with
+// the log-sum-exps of the CTA half that computed it.
 __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ AttnArgs a,
                                                       const __grid_constant__ CombineList cl) {
   const int i = blockIdx.x / TM, r = blockIdx.x % TM;
@@ -738,14 +736,16 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ At
   if (tg.row0 + r >= tg.rows_b) return;
   const int64_t grow = tg.grow0 + r;
   const int p0 = cl.piece0[i], p1 = cl.piece0[i + 1];
-  float mx = -INFINITY;
-  for (int p = p0; p < p1; ++p) mx = fmaxf(mx, a.ws_lse[(int64_t)p * TM + r]);
   const int d = threadIdx.x * 4;
+  const int half = d / HALF;                 // the CTA half these dims were computed in
+  const float* lse_h = a.ws_lse + half * TM + r;   // + p * 2 * TM: piece p
+  float mx = -INFINITY;
+  for (int p = p0; p < p1; ++p) mx = fmaxf(mx, lse_h[(int64_t)p * 2 * TM]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
   if (mx > -INFINITY) {
     for (int p = p0; p < p1; ++p) {
-      const float lp = a.ws_lse[(int64_t)p * TM + r];
+      const float lp = lse_h[(int64_t)p * 2 * TM];
       if (!(lp > -INFINITY)) continue;
       const float w = expf(lp - mx);
       wsum += w;
@@ -800,7 +800,7 @@ int cluster_slots() {
   return n;
 }
 
-size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc + 1) * sizeof(float); }
+size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc + 2) * sizeof(float); }
 
 }  // namespace
 

@@ -12,21 +12,26 @@
 #include "tc_ptx.cuh"
 #include "tmap.h"
 
+#include <mutex>
+
 namespace mla {
 namespace {
 
 using namespace tc;
 
-constexpr int GBM = 128, GBK = 64, GSTAGES = 4, GBN = 128;
+constexpr int GBM = 128, GBK = 64, GBN = 128;
 constexpr int GTHREADS = 192;
 constexpr int A_BYTES = GBM * GBK * 2;           // 16 KB
 constexpr int B_BYTES = GBN * GBK * 2;           // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int MAX_PAIRS = 512;                   // RoPE pairs with a table entry (d_R <= 1024)
 constexpr int STG_BYTES = 32 * 64;                // per epilogue warp: 32 rows x 32 cols bf16
-constexpr int OFF_TAB = GSTAGES * STAGE_BYTES + 256;
-constexpr int OFF_STG = OFF_TAB + MAX_PAIRS * 8;
-constexpr int GEMM_SMEM = OFF_STG + 4 * STG_BYTES + 1024;
+// Shared memory: the stage ring, barriers, the RoPE frequency table, epilogue staging.
+template <int ST> struct GLay {
+  static constexpr int OFF_TAB = ST * STAGE_BYTES + 256;
+  static constexpr int OFF_STG = OFF_TAB + MAX_PAIRS * 8;
+  static constexpr int SMEM = OFF_STG + 4 * STG_BYTES + 1024;
+};
 
 enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
 
@@ -44,7 +49,10 @@ struct TcGemm {
   unsigned int* err;
 };
 
-__global__ void __launch_bounds__(GTHREADS, 1)
+// GSTAGES-deep TMA ring.  Four stages (one CTA per SM) suit long K loops; two stages let
+// two CTAs share an SM, which hides the latency of short-K tiles (the absorption).
+template <int GSTAGES>
+__global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, TcGemm p) {
   extern __shared__ uint8_t smem_raw[];
@@ -56,7 +64,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   uint64_t* acce = accf + 2;                     // accumulator drained [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  double* inv_freq = reinterpret_cast<double*>(smem + OFF_TAB);
+  double* inv_freq = reinterpret_cast<double*>(smem + GLay<GSTAGES>::OFF_TAB);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nm = (p.M + GBM - 1) / GBM, nn = (p.N + GBN - 1) / GBN;
@@ -164,17 +172,32 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     const int r = (warp & 3) * 32 + lane;       // TMEM lane quarter = warp id % 4
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const Geo& G = p.geo;
-    uint8_t* stg = smem + OFF_STG + (warp - 2) * STG_BYTES;
+    uint8_t* stg = smem + GLay<GSTAGES>::OFF_STG + (warp - 2) * STG_BYTES;
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
       int m0, n0, z;
       tile_coords(t, m0, n0, z);
       const int acc = tc & 1;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[acc], (tc >> 1) & 1, abort, p.err,
-                                                         0x13, (r << 16) | tc));
-      tc_fence_after();
       const int64_t m = m0 + r;
       const bool row_ok = m < p.M;
+      // the absorption's share of RoPE(q_R) for this row: its loads are issued before the
+      // wait for the accumulator, so that their latency overlaps it and the drain
+      const bool rope_q = row_ok && p.mode == MODE_ABSORB && G.Dr > 0;
+      int qa0 = 0, qa1 = 0;
+      uint4 rin[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      const uint4* rsrc = nullptr;
+      if (rope_q) {
+        // the row's rotation pairs are shared out over the tiles of its row block, a
+        // multiple of 4 pairs (one 16-byte vector) each
+        const int nn = (p.N + GBN - 1) / GBN, npairs = G.Dr / 2;
+        const int ppt = ((npairs + nn - 1) / nn + 3) & ~3;
+        qa0 = (n0 / GBN) * ppt;
+        qa1 = qa0 + ppt < npairs ? qa0 + ppt : npairs;
+        rsrc = reinterpret_cast<const uint4*>(p.q_rope + (m * G.H + z) * G.Dr);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          if (qa0 / 4 + u < qa1 / 4) rin[u] = rsrc[qa0 / 4 + u];
+      }
       // this row's output base (element offset of column 0) and, for the cache, its token
       int64_t base = 0, g = 0;
       RopeAxes ax{0.0, 0.0, 0.0};
@@ -188,71 +211,78 @@ __global__ void __launch_bounds__(GTHREADS, 1)
       } else {
         base = (m * G.H + z) * G.Dn;
       }
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[acc], (tc >> 1) & 1, abort, p.err,
+                                                         0x13, (r << 16) | tc));
+      tc_fence_after();
       const uint32_t trow = tmem + lane_base + acc * GBN;
-      for (int c0 = 0; c0 < GBN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + c0, v);
+      // two 32-column TMEM loads in flight per wait
+      for (int c0 = 0; c0 < GBN; c0 += 64) {
+        uint32_t v[2][32];
+        tmem_ld32(trow + c0, v[0]);
+        tmem_ld32(trow + c0 + 32, v[1]);
         tmem_wait_ld();
-        if (c0 + 32 == GBN) {
+        if (c0 + 64 == GBN) {
           tc_fence_before();
           mbar_arrive(&acce[acc]);              // accumulator may be overwritten
         }
-        const int n = n0 + c0;                  // output column of v[0] (warp-uniform)
-        if (!ok || n >= p.N) continue;
-        float f[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-        if (p.mode == MODE_CACHE && n >= p.n_split && row_ok) {
+        for (int hh = 0; hh < 2; ++hh) {
+          const int n = n0 + c0 + 32 * hh;      // output column of v[hh][0] (warp-uniform)
+          if (!ok || n >= p.N) continue;
+          float f[32];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int q = (n + j - p.n_split) / 2;
-            rope_rotate_fast(f[j], f[j + 1], rope_axis_pos(G, ax, q), inv_freq[q]);
-          }
-        }
-        uint4* srow = reinterpret_cast<uint4*>(stg + lane * 64);
+          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[hh][j]);
+          if (p.mode == MODE_CACHE && n >= p.n_split && row_ok) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          srow[q ^ ((lane >> 1) & 3)] =
-              make_uint4(pack_bf16(f[8 * q + 0], f[8 * q + 1]), pack_bf16(f[8 * q + 2], f[8 * q + 3]),
-                         pack_bf16(f[8 * q + 4], f[8 * q + 5]), pack_bf16(f[8 * q + 6], f[8 * q + 7]));
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int rr = 8 * i + (lane >> 2), j = lane & 3;      // row of the warp, chunk
-          const int64_t rbase = __shfl_sync(0xffffffffu, base, rr);
-          if (m0 + (warp & 3) * 32 + rr < p.M) {
-            const uint4 w = reinterpret_cast<const uint4*>(stg + rr * 64)[j ^ ((rr >> 1) & 3)];
-            *reinterpret_cast<uint4*>(p.out + rbase + n + 8 * j) = w;
-          }
-        }
-        __syncwarp();
-      }
-      if (ok && row_ok && n0 == 0) {
-        if (p.mode == MODE_CACHE && p.slots) p.slots[m] = (int32_t)(g % G.S);
-        if (p.mode == MODE_ABSORB && G.Dr > 0) {
-          // q_abs[.., Dc:] = RoPE(q_R) for this tile's rows and head
-          const RopeAxes qa = rope_axes(G, p.first_tok + m % p.rows_per_batch);
-          const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + (m * G.H + z) * G.Dr);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (m * G.H + z) * G.row + G.Dc);
-          // 8 bf16 (4 pairs) per 16-byte vector; the loads of a chunk are issued together
-          for (int c = 0; c < G.Dr / 8; c += 4) {
-            uint4 in[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) in[u] = c + u < G.Dr / 8 ? src[c + u] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              if (c + u >= G.Dr / 8) break;
-              uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int q = (c + u) * 4 + e;
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                float a = f.x, b = f.y;
-                rope_rotate_fast(a, b, rope_axis_pos(G, qa, q), inv_freq[q]);
-                w[e] = pack_bf16(a, b);
-              }
-              dst[c + u] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int j = 0; j < 32; j += 2) {
+              const int q = (n + j - p.n_split) / 2;
+              rope_rotate_fast(f[j], f[j + 1], rope_axis_pos(G, ax, q), inv_freq[q]);
             }
+          }
+          uint4* srow = reinterpret_cast<uint4*>(stg + lane * 64);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            srow[q ^ ((lane >> 1) & 3)] = make_uint4(
+                pack_bf16(f[8 * q + 0], f[8 * q + 1]), pack_bf16(f[8 * q + 2], f[8 * q + 3]),
+                pack_bf16(f[8 * q + 4], f[8 * q + 5]), pack_bf16(f[8 * q + 6], f[8 * q + 7]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 8 * i + (lane >> 2), j = lane & 3;      // row of the warp, chunk
+            const int64_t rbase = __shfl_sync(0xffffffffu, base, rr);
+            if (m0 + (warp & 3) * 32 + rr < p.M) {
+              const uint4 w = reinterpret_cast<const uint4*>(stg + rr * 64)[j ^ ((rr >> 1) & 3)];
+              *reinterpret_cast<uint4*>(p.out + rbase + n + 8 * j) = w;
+            }
+          }
+          __syncwarp();
+        }
+      }
+      if (ok && row_ok && n0 == 0 && p.mode == MODE_CACHE && p.slots)
+        p.slots[m] = (int32_t)(g % G.S);
+      if (rope_q && ok && qa0 < qa1) {
+        // q_abs[.., Dc:] = RoPE(q_R) for the pairs [qa0, qa1) of this row
+        const RopeAxes qa = rope_axes(G, p.first_tok + m % p.rows_per_batch);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (m * G.H + z) * G.row + G.Dc);
+        for (int c = qa0 / 4; c < qa1 / 4; c += 2) {
+          uint4 in[2] = {rin[0], rin[1]};
+          if (c > qa0 / 4) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) if (c + u < qa1 / 4) in[u] = rsrc[c + u];
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (c + u >= qa1 / 4) break;
+            uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = (c + u) * 4 + e;
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+              float a = f.x, b = f.y;
+              rope_rotate_fast(a, b, rope_axis_pos(G, qa, q), inv_freq[q]);
+              w[e] = pack_bf16(a, b);
+            }
+            dst[c + u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
@@ -279,25 +309,42 @@ int sm_count() {
   return n;
 }
 
+template <int ST>
+cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
+                      const TcGemm& q, long long tiles, cudaStream_t st) {
+  {
+    // the shared-memory opt-in is per device
+    static std::mutex mu;
+    static uint64_t done = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 64 || !(done >> dev & 1)) {
+      e = cudaFuncSetAttribute(tc_gemm_kernel<ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               GLay<ST>::SMEM);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) done |= 1ull << dev;
+    }
+  }
+  const long long slots = (long long)sm_count() * (ST == 2 ? 2 : 1);
+  const int grid = (int)(tiles < slots ? tiles : slots);
+  if (grid == 0) return cudaSuccess;
+  tc_gemm_kernel<ST><<<grid, GTHREADS, GLay<ST>::SMEM, st>>>(A, B, B2, q);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launches(1);
+  return e;
+}
+
 cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
                    const TcGemm& p, int zcount, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
   TcGemm q = p;
   q.Z = zcount;
   const long long tiles =
       (long long)((p.M + GBM - 1) / GBM) * ((p.N + GBN - 1) / GBN) * zcount;
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  if (grid == 0) return cudaSuccess;
-  tc_gemm_kernel<<<grid, GTHREADS, GEMM_SMEM, st>>>(A, B, B2, q);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) count_launches(1);
-  return e;
+  // the absorption's tiles are two K-blocks long: two CTAs per SM hide their latency
+  if (p.mode == MODE_ABSORB) return launch_st<2>(A, B, B2, q, tiles, st);
+  return launch_st<4>(A, B, B2, q, tiles, st);
 }
 
 }  // namespace

@@ -324,6 +324,22 @@ def cpu_baseline(seconds: float = 12.0):
             "seconds": dt}
 
 
+def ranks_max(value: float, dist, device) -> float:
+    """The slowest rank's value (timings are max over ranks); the value itself when
+    there is no process group."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_step: float, steps: int, t_max_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_step * steps / (t_max_ms * 1e-3)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -358,25 +374,16 @@ def run_ours(args):
     launches = mla.mla_kernel_launches() - n0
     if world > 1:
         dist.barrier()
-    total_ms = sum(ms)
-    t_max = total_ms
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = ranks_max(sum(ms), dist if world > 1 else None, "cuda")
     # end to end through host buffers
     for _ in range(max(1, args.warmup // 2)):
         step.run_e2e()
     e2e_ms, _ = time_steps(torch, lambda a: step.run_e2e(), args.steps, flush)
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = ranks_max(sum(e2e_ms), dist if world > 1 else None, "cuda")
     fl = step_flops(wl)
     flops_step = sum(fl.values())
     ms_step = t_max / args.steps
-    value = world * flops_step * args.steps / (t_max * 1e-3) / 1e12
+    value = job_throughput(world, flops_step, args.steps, t_max) / 1e12
     peaks, peak_src = load_peaks()
     kernels_ms = {k: statistics.mean(v) for k, v in zip(Step.STAGES, parts)}
     att_ms = kernels_ms["attend"]
@@ -405,7 +412,7 @@ def run_ours(args):
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "traffic": None, "ms_per_launch": att_ms},
-            "e2e": {"value": world * flops_step * args.steps / (e2e_total * 1e-3) / 1e12,
+            "e2e": {"value": job_throughput(world, flops_step, args.steps, e2e_total) / 1e12,
                     "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(sum(v.nbytes for v in step.host.values())),
                     "d2h_bytes_per_step": int(step.out.numel() * 2),

@@ -1,0 +1,63 @@
+"""The N > 1 host logic of bench.py on CPU: two ranks over gloo (127.0.0.1).  Each rank
+runs its own replica, so the only exchange is the timing: every rank must end with the
+slowest rank's time, and the whole-job rate counts the units of all ranks.  The
+reference arm runs on rank 0 only; other ranks exit without work."""
+
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [7.0, 11.5][rank]              # the second rank is the slow one
+        t_max = bench.ranks_max(local_ms, dist, "cpu")
+        q.put((rank, t_max))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=5) for _ in range(2))
+    assert got == {0: 11.5, 1: 11.5}
+
+
+def test_job_throughput_counts_every_rank():
+    # 2 ranks x 3 steps x 10 units in 60 ms (slowest rank) = 1000 units/s
+    assert bench.job_throughput(2, 10.0, 3, 60.0) == pytest.approx(1000.0)
+    assert bench.ranks_max(3.0, None, "cpu") == 3.0
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""

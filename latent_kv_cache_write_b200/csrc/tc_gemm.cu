@@ -20,17 +20,21 @@ namespace {
 using namespace tc;
 
 constexpr int GBM = 128, GBK = 64, GBN = 128;
+
 constexpr int GTHREADS = 192;
 constexpr int A_BYTES = GBM * GBK * 2;           // 16 KB
 constexpr int B_BYTES = GBN * GBK * 2;           // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int MAX_PAIRS = 512;                   // RoPE pairs with a table entry (d_R <= 1024)
 constexpr int STG_BYTES = 32 * 64;                // per epilogue warp: 32 rows x 32 cols bf16
-// Shared memory: the stage ring, barriers, the RoPE frequency table, epilogue staging.
-template <int ST> struct GLay {
+constexpr int RB_BYTES = GBM * GBN * 4;          // split-K partial accumulator, 64 KB
+// Shared memory: the stage ring, barriers, the RoPE frequency table, epilogue staging and,
+// with split-K, the buffer the other CTA of the pair sends its fp32 partial tile into.
+template <int ST, bool SK> struct GLay {
   static constexpr int OFF_TAB = ST * STAGE_BYTES + 256;
   static constexpr int OFF_STG = OFF_TAB + MAX_PAIRS * 8;
-  static constexpr int SMEM = OFF_STG + 4 * STG_BYTES + 1024;
+  static constexpr int OFF_RB = OFF_STG + 4 * STG_BYTES;
+  static constexpr int SMEM = OFF_RB + (SK ? RB_BYTES : 0) + 1024;
 };
 
 enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
@@ -51,7 +55,12 @@ struct TcGemm {
 
 // GSTAGES-deep TMA ring.  Four stages (one CTA per SM) suit long K loops; two stages let
 // two CTAs share an SM, which hides the latency of short-K tiles (the absorption).
-template <int GSTAGES>
+// SPLITK: launched in clusters of two CTAs that share each tile, rank r taking half of
+// the K blocks; rank 1 sends its fp32 accumulator to rank 0 through distributed shared
+// memory (st.async, completion counted in bytes) and rank 0 adds it before the epilogue.
+// For few tiles with long K (the cache write: 65 tiles of K = 4096) it brings twice the
+// SMs' load bandwidth to the same tiles.
+template <int GSTAGES, bool SPLITK>
 __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, TcGemm p) {
@@ -62,14 +71,23 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
   uint64_t* empty = full + GSTAGES;
   uint64_t* accf = empty + GSTAGES;              // accumulator ready [2]
   uint64_t* acce = accf + 2;                     // accumulator drained [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* rbf = acce + 2;                      // split-K: partial landed (rank 0, tx bytes)
+  uint64_t* rbe = acce + 3;                      // split-K: rank 0 has read it (rank 1)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 4);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  double* inv_freq = reinterpret_cast<double*>(smem + GLay<GSTAGES>::OFF_TAB);
+  using GL = GLay<GSTAGES, SPLITK>;
+  double* inv_freq = reinterpret_cast<double*>(smem + GL::OFF_TAB);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nm = (p.M + GBM - 1) / GBM, nn = (p.N + GBN - 1) / GBN;
   const int ntiles = nm * nn * p.Z;
   const int nk = (p.K + GBK - 1) / GBK;
+  // tiles this CTA (or CTA pair) walks, and its K blocks
+  const uint32_t crank = SPLITK ? cluster_ctarank() : 0u;
+  const int t_first = SPLITK ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int t_step = SPLITK ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int kb0 = SPLITK && crank ? nk / 2 : 0;
+  const int kb1 = SPLITK && !crank ? nk / 2 : nk;
 
   if (tid == 0) {
     for (int s = 0; s < GSTAGES; ++s) {
@@ -80,6 +98,8 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], 128);
     }
+    mbar_init(rbf, 1);
+    mbar_init(rbe, 1);
     *abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
@@ -94,6 +114,7 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     inv_freq[q] = rope_inv_freq(p.geo, q);
   tc_fence_before();
   __syncthreads();
+  if constexpr (SPLITK) cluster_sync();        // the pair's barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -108,13 +129,13 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      for (int t = t_first; t < ntiles; t += t_step) {
         int m0, n0, z;
         tile_coords(t, m0, n0, z);
         const bool second = p.mode == MODE_CACHE && n0 >= p.n_split;
         const CUtensorMap* mB = second ? &tmB2 : &tmB;
         const int nb = second ? n0 - p.n_split : n0;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % GSTAGES;
           if (!mbar_wait(&empty[s], ((it / GSTAGES) & 1) ^ 1, abort, p.err, 0x11, kb)) break;
           uint8_t* a = smem + s * STAGE_BYTES;
@@ -136,12 +157,12 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(GBM, GBN, false, p.b_mn != 0);
       uint32_t it = 0, tc = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+      for (int t = t_first; t < ntiles; t += t_step, ++tc) {
         const int acc = tc & 1;
         if (!mbar_wait(&acce[acc], ((tc >> 1) & 1) ^ 1, abort, p.err, 0x14, tc)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * GBN;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % GSTAGES;
           if (!mbar_wait(&full[s], (it / GSTAGES) & 1, abort, p.err, 0x12, kb)) break;
           tc_fence_after();
@@ -154,7 +175,8 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
             // K-major operands advance 32 bytes per 16-element K step inside the swizzle
             // atom; the MN-major B advances 16 rows of 128 bytes.
             const uint64_t bstep = p.b_mn ? (uint64_t)(ks * 2048 >> 4) : (uint64_t)(ks * 32 >> 4);
-            mma_ss(d, da + (uint64_t)(ks * 32 >> 4), db + bstep, idesc, (kb | ks) != 0);
+            mma_ss(d, da + (uint64_t)(ks * 32 >> 4), db + bstep, idesc,
+                   (kb != kb0 || ks != 0) ? 1u : 0u);
           }
           mma_commit(&empty[s]);
         }
@@ -172,12 +194,48 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     const int r = (warp & 3) * 32 + lane;       // TMEM lane quarter = warp id % 4
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const Geo& G = p.geo;
-    uint8_t* stg = smem + GLay<GSTAGES>::OFF_STG + (warp - 2) * STG_BYTES;
+    uint8_t* stg = smem + GL::OFF_STG + (warp - 2) * STG_BYTES;
+    // split-K partial tile, chunk-major [32 chunks of 4 floats][128 rows]: conflict-free
+    // for both the sending and the reading thread of a row
+    const float4* rb = reinterpret_cast<const float4*>(smem + GL::OFF_RB) + r;
     uint32_t tc = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+    for (int t = t_first; t < ntiles; t += t_step, ++tc) {
       int m0, n0, z;
       tile_coords(t, m0, n0, z);
       const int acc = tc & 1;
+      if constexpr (SPLITK) {
+        if (crank == 1) {
+          // drain this CTA's half-K accumulator into rank 0's buffer once rank 0 has read
+          // the previous tile's
+          bool okr = __all_sync(0xffffffffu, mbar_wait(&accf[acc], (tc >> 1) & 1, abort, p.err,
+                                                         0x15, (r << 16) | tc));
+          if (okr)
+            okr = __all_sync(0xffffffffu, mbar_wait_cluster(rbe, (tc & 1) ^ 1, abort, p.err,
+                                                             0x16, (r << 16) | tc));
+          tc_fence_after();
+          const uint32_t trow = tmem + lane_base + acc * GBN;
+          const uint32_t dst = mapa(smem_u32(smem + GL::OFF_RB), 0) + (uint32_t)r * 16;
+          const uint32_t dbar = mapa(smem_u32(rbf), 0);
+          for (int c0 = 0; c0 < GBN; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(trow + c0, v);
+            tmem_wait_ld();
+            if (c0 + 32 == GBN) {
+              tc_fence_before();
+              mbar_arrive(&acce[acc]);          // accumulator may be overwritten
+            }
+            if (!okr) continue;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              st_async_v4(dst + (uint32_t)(c0 / 4 + q) * (GBM * 16), v[4 * q], v[4 * q + 1],
+                          v[4 * q + 2], v[4 * q + 3], dbar);
+          }
+          if (!okr) break;
+          continue;
+        }
+        // rank 0: the partial of this tile lands in its buffer (armed here, per tile)
+        if (r == 0) mbar_expect_tx(rbf, RB_BYTES);
+      }
       const int64_t m = m0 + r;
       const bool row_ok = m < p.M;
       // the absorption's share of RoPE(q_R) for this row: its loads are issued before the
@@ -211,8 +269,13 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
       } else {
         base = (m * G.H + z) * G.Dn;
       }
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[acc], (tc >> 1) & 1, abort, p.err,
-                                                         0x13, (r << 16) | tc));
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[acc], (tc >> 1) & 1, abort, p.err,
+                                                   0x13, (r << 16) | tc));
+      if constexpr (SPLITK) {
+        if (ok)
+          ok = __all_sync(0xffffffffu, mbar_wait_cluster(rbf, tc & 1, abort, p.err, 0x17,
+                                                         (r << 16) | tc));
+      }
       tc_fence_after();
       const uint32_t trow = tmem + lane_base + acc * GBN;
       // two 32-column TMEM loads in flight per wait
@@ -232,6 +295,17 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
           float f[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[hh][j]);
+          if constexpr (SPLITK) {
+            // plus the other half of K, from the pair's rank 1
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 o = rb[((c0 + 32 * hh) / 4 + q) * GBM];
+              f[4 * q] += o.x;
+              f[4 * q + 1] += o.y;
+              f[4 * q + 2] += o.z;
+              f[4 * q + 3] += o.w;
+            }
+          }
           if (p.mode == MODE_CACHE && n >= p.n_split && row_ok) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
@@ -257,6 +331,11 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
           }
           __syncwarp();
         }
+      }
+      if constexpr (SPLITK) {
+        // every row of the partial is read: rank 1 may send the next tile's
+        named_bar(1, 128);
+        if (r == 0) mbar_arrive_cluster_relaxed(mapa(smem_u32(rbe), 1));
       }
       if (ok && row_ok && n0 == 0 && p.mode == MODE_CACHE && p.slots)
         p.slots[m] = (int32_t)(g % G.S);
@@ -292,6 +371,7 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if constexpr (SPLITK) cluster_sync();        // no remote access into this CTA is pending
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 2 * GBN);
@@ -309,9 +389,10 @@ int sm_count() {
   return n;
 }
 
-template <int ST>
+template <int ST, bool SK>
 cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
                       const TcGemm& q, long long tiles, cudaStream_t st) {
+  using GL = GLay<ST, SK>;
   {
     // the shared-memory opt-in is per device
     static std::mutex mu;
@@ -321,16 +402,37 @@ cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
     if (dev >= 64 || !(done >> dev & 1)) {
-      e = cudaFuncSetAttribute(tc_gemm_kernel<ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               GLay<ST>::SMEM);
+      e = cudaFuncSetAttribute(tc_gemm_kernel<ST, SK>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, GL::SMEM);
       if (e != cudaSuccess) return e;
       if (dev < 64) done |= 1ull << dev;
     }
   }
-  const long long slots = (long long)sm_count() * (ST == 2 ? 2 : 1);
-  const int grid = (int)(tiles < slots ? tiles : slots);
-  if (grid == 0) return cudaSuccess;
-  tc_gemm_kernel<ST><<<grid, GTHREADS, GLay<ST>::SMEM, st>>>(A, B, B2, q);
+  if (!SK) {
+    const long long slots = (long long)sm_count() * (ST == 2 ? 2 : 1);
+    const int grid = (int)(tiles < slots ? tiles : slots);
+    if (grid == 0) return cudaSuccess;
+    tc_gemm_kernel<ST, SK><<<grid, GTHREADS, GL::SMEM, st>>>(A, B, B2, q);
+  } else {
+    // clusters of two CTAs, one cluster per tile up to one per SM pair
+    const long long pairs = sm_count() / 2;
+    const int nclu = (int)(tiles < pairs ? tiles : pairs);
+    if (nclu == 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * nclu);
+    cfg.blockDim = dim3(GTHREADS);
+    cfg.dynamicSmemBytes = GL::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<ST, SK>, A, B, B2, q);
+    if (e != cudaSuccess) return e;
+  }
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;
@@ -342,9 +444,13 @@ cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap
   q.Z = zcount;
   const long long tiles =
       (long long)((p.M + GBM - 1) / GBM) * ((p.N + GBN - 1) / GBN) * zcount;
+  const int nk = (p.K + GBK - 1) / GBK;
   // the absorption's tiles are two K-blocks long: two CTAs per SM hide their latency
-  if (p.mode == MODE_ABSORB) return launch_st<2>(A, B, B2, q, tiles, st);
-  return launch_st<4>(A, B, B2, q, tiles, st);
+  if (p.mode == MODE_ABSORB) return launch_st<2, false>(A, B, B2, q, tiles, st);
+  // fewer tiles than SMs and a long K loop (the cache write): split K over CTA pairs
+  if (p.mode == MODE_CACHE && nk >= 2 && tiles < sm_count())
+    return launch_st<4, true>(A, B, B2, q, tiles, st);
+  return launch_st<4, false>(A, B, B2, q, tiles, st);
 }
 
 }  // namespace

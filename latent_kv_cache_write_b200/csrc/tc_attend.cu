@@ -247,18 +247,22 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
 }
 
 // Q latent half of row `grow` -> TMEM columns from `tq` (A operand of the score MMA),
-// bf16 pairs per column; each warpgroup loads half of the row.
+// bf16 pairs per column; each warpgroup loads half of the row.  All 16 vector loads are
+// issued before the first TMEM store, so their latencies overlap.
 __device__ __forceinline__ void load_q(const AttnArgs& a, uint32_t tq, int64_t grow,
                                        bool row_ok, uint32_t rank, int wg) {
   const uint4* src = reinterpret_cast<const uint4*>(a.q_abs + grow * a.g.row + rank * HALF +
                                                     wg * (HALF / 2));
-#pragma unroll 1
+  uint4 x[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) x[q] = row_ok ? src[q] : make_uint4(0, 0, 0, 0);
+#pragma unroll
   for (int c = 0; c < HALF / 64; ++c) {
     uint32_t v[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      uint4 x = row_ok ? src[c * 4 + q] : make_uint4(0, 0, 0, 0);
-      v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+      v[4 * q] = x[4 * c + q].x; v[4 * q + 1] = x[4 * c + q].y;
+      v[4 * q + 2] = x[4 * c + q].z; v[4 * q + 3] = x[4 * c + q].w;
     }
     tmem_st16(tq + wg * (HALF / 4) + c * 16, v);
   }
@@ -465,6 +469,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int64_t k_end_row =
           key_end(G, a.q_first, a.k_first + a.n_keys, row_valid ? r_in_b / G.H : tg.i_last);
       const int n = sw.nb();
+      {
+        // the next segment's Q rows (this CTA's latent half, this warpgroup's half of it)
+        // into L2 now, so that their load into TMEM at the segment's end is short
+        SegWalk nx = sw;
+        nx.next(a);
+        if (nx.valid() && nx.tg.row0 + t < nx.tg.rows_b) {
+          const char* qrow = reinterpret_cast<const char*>(
+              a.q_abs + (nx.tg.grow0 + t) * G.row + rank * HALF + wg * (HALF / 2));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128));
+        }
+      }
       float m_last = -INFINITY, l = 0.f;       // this warpgroup's running sum and its max
       for (int jl = wg; jl < n; jl += 2) {
         const int j = sw.jb + jl;              // block of the tile

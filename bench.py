@@ -324,6 +324,25 @@ def cpu_baseline(seconds: float = 12.0):
             "seconds": dt}
 
 
+# DRAM bytes (read + write) of one chunk attention launch, from the ncu capture summarised in
+# profiles/attend_kernel_video_chunk.md.  Counters describe the kernel source they were
+# taken on: the value is reported only while that source is unchanged.
+ATTEND_TRAFFIC = {"bytes": 73_488_384 + 32_379_136,
+                  "source": "latent_kv_cache_write_b200/csrc/tc_attend.cu",
+                  "sha256": "04cfb0a9b3a0f490168e311e044c6643184007c907ad195918a34e09e85b63c8"}
+
+
+def attend_traffic():
+    import hashlib
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), ATTEND_TRAFFIC["source"])
+    try:
+        with open(path, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return ATTEND_TRAFFIC["bytes"] if digest == ATTEND_TRAFFIC["sha256"] else None
+
+
 def ranks_max(value: float, dist, device) -> float:
     """The slowest rank's value (timings are max over ranks); the value itself when
     there is no process group."""
@@ -411,7 +430,8 @@ def run_ours(args):
             "roofline": {"kernel": "mla_attend", "bound": "tensor", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "traffic": None, "ms_per_launch": att_ms},
+                         "traffic": attend_traffic(), "traffic_unit": "B per launch (ncu)",
+                         "ms_per_launch": att_ms},
             "e2e": {"value": job_throughput(world, flops_step, args.steps, e2e_total) / 1e12,
                     "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(sum(v.nbytes for v in step.host.values())),

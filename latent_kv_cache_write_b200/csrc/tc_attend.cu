@@ -36,6 +36,7 @@
 // Warp roles (352 threads): warps 0-3 and 4-7 are the two softmax warpgroups (thread =
 // row = TMEM lane), warp 8 is the TMA producer, warp 9 issues the score MMAs, loads the
 // Q RoPE tiles and owns the TMEM allocation, warp 10 issues the PV MMAs.
+#include "attend_common.cuh"
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tmap.h"
@@ -49,10 +50,8 @@ namespace mla {
 namespace {
 
 using namespace tc;
+using namespace attn;
 
-constexpr int TM = 128;                               // rows per tile
-constexpr int BN = 64;                                // keys per block
-constexpr int HALF = 256;                             // latent dims per CTA
 constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
 constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB of latent per stage
 constexpr int RBOX_BYTES = BN * 32 * 2;               // 64 keys x 32 RoPE dims, 4 KB
@@ -62,7 +61,6 @@ constexpr int QR_BYTES = TM * 32 * 2;                 // this CTA's Q RoPE part,
 // [8 x 16 B][128 rows].  P buffer of a warpgroup, 16 KB: bf16, 128-byte swizzled rows.
 constexpr int XP_BYTES = TM * BN * 2;
 constexpr int NTHREADS = 352;
-constexpr int MAXC = 128;                             // clusters one launch can schedule
 
 // Shared-memory layout and barriers of the two pipeline depths.
 //   DEEP = false: 4 K/V stages; separate exchange and P buffers; an exchange buffer is
@@ -111,19 +109,6 @@ struct Lay {
 constexpr uint32_t O_COL = 0, Q_COL = 256, S_COL = 384;
 constexpr unsigned FULL = 0xffffffffu;
 
-struct AttnArgs {
-  Geo g;
-  int64_t n_q, q_first, k_first, n_keys;
-  float scale_log2;
-  const bf16* q_abs;
-  bf16* o_lat;
-  float* lse;
-  float* ws_o;              // partial outputs [slot][TM][Dc], fp32, normalised by their l
-  float* ws_lse;            // their natural log-sum-exps, one per CTA half [slot][2][TM]
-  int tiles_per_batch;
-  unsigned int* err;
-};
-
 // Cluster c walks the key blocks from (cut_tile[c], cut_blk[c]) up to, not including,
 // (cut_tile[c + 1], cut_blk[c + 1]) in tile-major order; its partial segments take the
 // workspace slots slot0[c], slot0[c] + 1, ...
@@ -132,62 +117,6 @@ struct Sched {
   int32_t cut_blk[MAXC + 1];
   int32_t slot0[MAXC];
 };
-
-// Key blocks of one tile: its rows see the keys k_first .. k_first + L - 1 (frame-
-// block-causal bound of its last row), stored in the ring as two contiguous slot runs.
-struct Blocks {
-  int64_t k_first, p1, n1, L;
-  int nb1, nblk;
-  // block j: first ring slot, first global token, number of keys
-  __device__ void get(int j, int64_t& slot0, int64_t& g0, int& valid) const {
-    if (j < nb1) {
-      slot0 = p1 + (int64_t)j * BN;
-      g0 = k_first + (int64_t)j * BN;
-      const int64_t v = n1 - (int64_t)j * BN;
-      valid = v < BN ? (int)v : BN;
-    } else {
-      const int64_t jj = j - nb1;
-      slot0 = jj * BN;
-      g0 = k_first + n1 + jj * BN;
-      const int64_t v = L - n1 - jj * BN;
-      valid = v < BN ? (int)v : BN;
-    }
-  }
-};
-
-struct TileGeo {
-  int b;
-  int64_t rows_b, row0, grow0, i_last;
-  Blocks blk;
-};
-
-// one past the last key query i sees (frame-block-causal, clipped to the key window)
-__host__ __device__ inline int64_t key_end(const Geo& G, int64_t q_first, int64_t k_lim,
-                                           int64_t i) {
-  const int64_t e = ((q_first + i) / G.F + 1) * G.F;
-  return e < k_lim ? e : k_lim;
-}
-
-__host__ __device__ inline TileGeo tile_geo(const Geo& G, int64_t n_q, int64_t q_first,
-                                            int64_t k_first, int64_t n_keys,
-                                            int tiles_per_batch, int tile) {
-  TileGeo t;
-  t.b = tile / tiles_per_batch;
-  const int tb = tile - t.b * tiles_per_batch;
-  t.rows_b = n_q * G.H;
-  t.row0 = (int64_t)tb * TM;
-  t.grow0 = (int64_t)t.b * t.rows_b + t.row0;
-  const int64_t last_row = (t.row0 + TM < t.rows_b ? t.row0 + TM : t.rows_b) - 1;
-  t.i_last = last_row / G.H;
-  Blocks& k = t.blk;
-  k.k_first = k_first;
-  k.L = key_end(G, q_first, k_first + n_keys, t.i_last) - k_first;
-  k.p1 = k_first % G.S;
-  k.n1 = k.L < G.S - k.p1 ? k.L : G.S - k.p1;
-  k.nb1 = (int)((k.n1 + BN - 1) / BN);
-  k.nblk = k.nb1 + (int)((k.L - k.n1 + BN - 1) / BN);
-  return t;
-}
 
 // The segments of one cluster's range, in order.  Every role walks the same sequence
 // and keeps the running counts that barrier phases and ring stages derive from.
@@ -733,54 +662,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// Split tiles to merge: tile[i] has the partial segments in workspace slots
-// [piece0[i], piece0[i + 1]).
-struct CombineList {
-  int32_t n;
-  int32_t tile[MAXC];
-  int32_t piece0[MAXC + 1];
-};
-
-// One CTA per (split tile, row), 4 latent dims per thread: the output is the partials
-// weighted by exp(lse_p - lse), lse = log sum_p exp(lse_p), each half of the dims with
-// the log-sum-exps of the CTA half that computed it.
-__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ AttnArgs a,
-                                                      const __grid_constant__ CombineList cl) {
-  const int i = blockIdx.x / TM, r = blockIdx.x % TM;
-  const TileGeo tg =
-      tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, cl.tile[i]);
-  if (tg.row0 + r >= tg.rows_b) return;
-  const int64_t grow = tg.grow0 + r;
-  const int p0 = cl.piece0[i], p1 = cl.piece0[i + 1];
-  const int d = threadIdx.x * 4;
-  const int half = d / HALF;                 // the CTA half these dims were computed in
-  const float* lse_h = a.ws_lse + half * TM + r;   // + p * 2 * TM: piece p
-  float mx = -INFINITY;
-  for (int p = p0; p < p1; ++p) mx = fmaxf(mx, lse_h[(int64_t)p * 2 * TM]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
-  if (mx > -INFINITY) {
-    for (int p = p0; p < p1; ++p) {
-      const float lp = lse_h[(int64_t)p * 2 * TM];
-      if (!(lp > -INFINITY)) continue;
-      const float w = expf(lp - mx);
-      wsum += w;
-      const float4 o =
-          *reinterpret_cast<const float4*>(a.ws_o + ((int64_t)p * TM + r) * a.g.Dc + d);
-      acc.x += w * o.x;
-      acc.y += w * o.y;
-      acc.z += w * o.z;
-      acc.w += w * o.w;
-    }
-  }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  uint2 out;
-  out.x = pack_bf16(acc.x * inv, acc.y * inv);
-  out.y = pack_bf16(acc.z * inv, acc.w * inv);
-  *reinterpret_cast<uint2*>(a.o_lat + grow * a.g.Dc + d) = out;
-  if (threadIdx.x == 0 && a.lse) a.lse[grow] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
-}
-
 // Clusters of the attention kernel that can be resident at once on the current device
 // (one CTA per SM; a cluster needs two SMs of one GPC), capped at MAXC.  The first call
 // on a device also opts the kernel in to its shared memory.  0 on failure.
@@ -939,8 +820,7 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   if (e != cudaSuccess) return e;
   count_launches(1);
   if (cl.n > 0) {
-    combine_kernel<<<(unsigned)(cl.n * TM), 128, 0, st>>>(a, cl);
-    e = cudaGetLastError();
+    e = launch_combine(a, cl, st);
     if (e != cudaSuccess) return e;
     count_launches(1);
   }

@@ -747,34 +747,58 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     pre[t + 1] = pre[t] + nbt[t];
   }
   const int64_t W = pre[T];
-  Sched sc{};
-  int G;
-  if (split && W > 0) {
-    // cut c at block W*c/G; tiles without blocks go with the range before them
-    G = (int)(W < ncl ? W : ncl);
-    int t = 0;
-    for (int c = 1; c <= G; ++c) {
-      const int64_t pos = W * c / G;
-      while (t < T && pre[t + 1] <= pos) ++t;      // tile holding block `pos`
-      sc.cut_tile[c] = t;
-      sc.cut_blk[c] = t < T ? (int)(pos - pre[t]) : 0;
+  // Two candidate schedules, costed in key blocks: a cluster's blocks plus SEG_COST per
+  // segment it walks (the switch: Q reload, output epilogue, pipeline refill), plus
+  // COMBINE_COST when tiles are split (the merge launch).  Both costs were measured on
+  // B200 (video chunk, long window and decode shapes).
+  constexpr int64_t SEG_COST = 7, COMBINE_COST = 16;
+  auto cost = [&](const Sched& c, int nc) {
+    int64_t worst = 0;
+    bool any_split = false;
+    for (int k = 0; k < nc; ++k) {
+      const int t0 = c.cut_tile[k], b0 = c.cut_blk[k], t1 = c.cut_tile[k + 1], b1 = c.cut_blk[k + 1];
+      const int64_t blocks = (pre[t1] + b1) - (pre[t0] + b0);
+      const int64_t segs = (int64_t)(t1 - t0) + (b1 > 0 ? 1 : 0);
+      any_split = any_split || b0 > 0 || b1 > 0;
+      worst = blocks + SEG_COST * segs > worst ? blocks + SEG_COST * segs : worst;
     }
-  } else {
-    // cuts on tile boundaries: the first one at or past an equal share of the blocks
-    // (of the tiles when there are no blocks)
-    G = T < ncl ? T : ncl;
+    return worst + (any_split ? COMBINE_COST : 0);
+  };
+  // cuts on tile boundaries: the first one at or past an equal share of the blocks (of the
+  // tiles when there are no blocks)
+  Sched whole{};
+  const int G_whole = T < ncl ? T : ncl;
+  {
     int t = 0;
-    for (int c = 1; c <= G; ++c) {
-      if (c == G) {
+    for (int c = 1; c <= G_whole; ++c) {
+      if (c == G_whole) {
         t = T;
       } else if (W > 0) {
-        const int64_t pos = W * c / G;
+        const int64_t pos = W * c / G_whole;
         while (t < T && pre[t] < pos) ++t;
       } else {
-        t = (int)((int64_t)T * c / G);
+        t = (int)((int64_t)T * c / G_whole);
       }
-      sc.cut_tile[c] = t;
-      sc.cut_blk[c] = 0;
+      whole.cut_tile[c] = t;
+      whole.cut_blk[c] = 0;
+    }
+  }
+  Sched sc = whole;
+  int G = G_whole;
+  if (split && W > 0) {
+    // cut c at block W*c/G; tiles without blocks go with the range before them
+    Sched sk{};
+    const int G_split = (int)(W < ncl ? W : ncl);
+    int t = 0;
+    for (int c = 1; c <= G_split; ++c) {
+      const int64_t pos = W * c / G_split;
+      while (t < T && pre[t + 1] <= pos) ++t;      // tile holding block `pos`
+      sk.cut_tile[c] = t;
+      sk.cut_blk[c] = t < T ? (int)(pos - pre[t]) : 0;
+    }
+    if (cost(sk, G_split) < cost(whole, G_whole)) {
+      sc = sk;
+      G = G_split;
     }
   }
   sc.cut_tile[0] = 0;

@@ -204,6 +204,7 @@ def test_single_frame_window_and_last_query(cuda_ok):
 
 
 def _attend(r, wl, use_ws):
+    """mla_attend with or without a workspace; returns (o_lat, lse, kernels launched)."""
     import latent_kv_cache_write_b200 as mla
     T = wl.n_queries
     o = torch.empty((wl.batch, T, wl.n_heads, wl.d_latent), dtype=torch.bfloat16, device=P.DEV)
@@ -212,38 +213,63 @@ def _attend(r, wl, use_ws):
     if use_ws:
         nws = mla.mla_attend_workspace_size(r.shape, T, wl.n_keys)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=P.DEV)
+    n0 = mla.mla_kernel_launches()
     mla.mla_attend(r.shape, r.q_abs, T, wl.q_first_tok, r.cache, wl.k_first_tok, wl.n_keys,
                    wl.softmax_scale, o, lse, ws, nws)
+    launches = mla.mla_kernel_launches() - n0
     torch.cuda.synchronize()
     assert mla.mla_device_error() == 0
-    return P.download(o), lse.cpu().numpy()
+    return P.download(o), lse.cpu().numpy(), launches
 
 
-@pytest.mark.parametrize("use_ws", [True, False], ids=["split_keys", "whole_tiles"])
-def test_schedule_many_segments(cuda_ok, use_ws):
-    """136 tiles of 5 key blocks: more blocks than SM pairs, so every cluster walks
-    several segments (tile switches inside one launch); with a workspace the cuts also
-    split tiles (partials merged by the combine kernel), without one they fall on tile
-    boundaries.  All rows against the oracle."""
-    wl = C.small_variant(C.VIDEO_CHUNK).scaled(name="video_chunk_sched", batch=8,
-                                               n_heads=32, chunk_frames=1)
+# Shapes on which the schedule splits tiles (the host prefers it when the balance it buys
+# outweighs the extra segment switches and the merge launch): many key blocks per tile,
+# about as many tiles as SM pairs, so each cluster walks several segments.
+SPLIT_CHUNK = C.small_variant(C.VIDEO_CHUNK).scaled(
+    name="video_chunk_split", batch=5, n_heads=32, chunk_frames=1, window_frames=38,
+    first_chunk_frame=38, ring_slots=39 * 66)
+SPLIT_DECODE = C.small_variant(C.DECODE).scaled(
+    name="decode_split", batch=8, ring_slots=4096, window_frames=4095, first_chunk_frame=4095)
+
+
+@pytest.mark.parametrize("wl", [SPLIT_CHUNK, SPLIT_DECODE], ids=lambda w: w.name)
+@pytest.mark.parametrize("use_ws", [True, False], ids=["workspace", "no_workspace"])
+def test_schedule_split_and_whole(cuda_ok, wl, use_ws):
+    """With a workspace these shapes cut tiles between clusters (the merge kernel runs:
+    two launches); without one the cuts fall on tile boundaries (one launch).  Every
+    cluster walks several segments (tile switches inside one launch).  All rows against
+    the oracle."""
     r = P.run_chunk(P.populate(wl, seed=5))
     lat_ref, lse_ref = O.attend_latent(P.download(r.q_abs), P.download(r.cache), wl.q_first_tok,
                                        wl.k_first_tok, wl.n_keys, wl.softmax_scale, wl)
-    o, lse = _attend(r, wl, use_ws)
+    o, lse, launches = _attend(r, wl, use_ws)
+    assert launches == (2 if use_ws else 1)
     P.tol_check(o, lat_ref, wl.dtype, "o_lat")
     np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=2e-2)
 
 
+def test_schedule_many_whole_tiles(cuda_ok):
+    """136 short tiles (5 key blocks each) on fewer SM pairs: whole-tile segments, several
+    per cluster, with or without a workspace."""
+    wl = C.small_variant(C.VIDEO_CHUNK).scaled(name="video_chunk_sched", batch=8,
+                                               n_heads=32, chunk_frames=1)
+    r = P.run_chunk(P.populate(wl, seed=5))
+    lat_ref, _ = O.attend_latent(P.download(r.q_abs), P.download(r.cache), wl.q_first_tok,
+                                 wl.k_first_tok, wl.n_keys, wl.softmax_scale, wl)
+    for use_ws in (True, False):
+        o, _, launches = _attend(r, wl, use_ws)
+        assert launches == 1
+        P.tol_check(o, lat_ref, wl.dtype, "o_lat")
+
+
 def test_schedule_split_matches_whole(cuda_ok):
-    """The split-key and the whole-tile schedules give the same attention (up to the
-    rounding of the partial merge) on the full decode shape, where 64 tiles are fewer
-    than the SM pairs."""
-    wl = C.DECODE
-    r = P.populate(wl, seed=2)
-    r = P.run_chunk(r, with_lse=False)
-    o1, l1 = _attend(r, wl, True)
-    o2, l2 = _attend(r, wl, False)
+    """The split-key and the whole-tile schedules give the same attention, up to the
+    rounding of the partial merge."""
+    wl = SPLIT_DECODE
+    r = P.run_chunk(P.populate(wl, seed=2), with_lse=False)
+    o1, l1, n1 = _attend(r, wl, True)
+    o2, l2, n2 = _attend(r, wl, False)
+    assert (n1, n2) == (2, 1)
     err = float(np.linalg.norm(o1 - o2) / np.linalg.norm(o2))
     assert err <= 4e-3, err
     np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-3)

@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(32 * CROWS) combine_kernel(const __grid_consta
   const int r = (blockIdx.x % (TM / CROWS)) * CROWS + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const TileGeo tg =
-      tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, cl.tile[i]);
+      tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, cl.tile[i], a.bn);
   if (tg.row0 + r >= tg.rows_b) return;
   const int64_t grow = tg.grow0 + r;
   const int p0 = cl.piece0[i], p1 = cl.piece0[i + 1];

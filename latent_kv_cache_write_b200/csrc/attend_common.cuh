@@ -8,7 +8,6 @@ namespace mla {
 namespace attn {
 
 constexpr int TM = 128;                               // rows per tile
-constexpr int BN = 64;                                // keys per block
 constexpr int HALF = 256;                             // latent dims per CTA of a cluster
 constexpr int MAXC = 128;                             // clusters one launch can schedule
 
@@ -22,6 +21,7 @@ struct AttnArgs {
   float* ws_o;              // partial outputs [slot][TM][Dc], fp32, normalised by their l
   float* ws_lse;            // their natural log-sum-exps, one per CTA half [slot][2][TM]
   int tiles_per_batch;
+  int bn;                   // keys per block of the launch
   unsigned int* err;
 };
 
@@ -29,20 +29,21 @@ struct AttnArgs {
 // block-causal bound of its last row), stored in the ring as two contiguous slot runs.
 struct Blocks {
   int64_t k_first, p1, n1, L;
+  int bn;                   // keys per block
   int nb1, nblk;
   // block j: first ring slot, first global token, number of keys
   __device__ void get(int j, int64_t& slot0, int64_t& g0, int& valid) const {
     if (j < nb1) {
-      slot0 = p1 + (int64_t)j * BN;
-      g0 = k_first + (int64_t)j * BN;
-      const int64_t v = n1 - (int64_t)j * BN;
-      valid = v < BN ? (int)v : BN;
+      slot0 = p1 + (int64_t)j * bn;
+      g0 = k_first + (int64_t)j * bn;
+      const int64_t v = n1 - (int64_t)j * bn;
+      valid = v < bn ? (int)v : bn;
     } else {
       const int64_t jj = j - nb1;
-      slot0 = jj * BN;
-      g0 = k_first + n1 + jj * BN;
-      const int64_t v = L - n1 - jj * BN;
-      valid = v < BN ? (int)v : BN;
+      slot0 = jj * bn;
+      g0 = k_first + n1 + jj * bn;
+      const int64_t v = L - n1 - jj * bn;
+      valid = v < bn ? (int)v : bn;
     }
   }
 };
@@ -62,7 +63,7 @@ __host__ __device__ inline int64_t key_end(const Geo& G, int64_t q_first, int64_
 
 __host__ __device__ inline TileGeo tile_geo(const Geo& G, int64_t n_q, int64_t q_first,
                                             int64_t k_first, int64_t n_keys,
-                                            int tiles_per_batch, int tile) {
+                                            int tiles_per_batch, int tile, int bn) {
   TileGeo t;
   t.b = tile / tiles_per_batch;
   const int tb = tile - t.b * tiles_per_batch;
@@ -76,8 +77,9 @@ __host__ __device__ inline TileGeo tile_geo(const Geo& G, int64_t n_q, int64_t q
   k.L = key_end(G, q_first, k_first + n_keys, t.i_last) - k_first;
   k.p1 = k_first % G.S;
   k.n1 = k.L < G.S - k.p1 ? k.L : G.S - k.p1;
-  k.nb1 = (int)((k.n1 + BN - 1) / BN);
-  k.nblk = k.nb1 + (int)((k.L - k.n1 + BN - 1) / BN);
+  k.bn = bn;
+  k.nb1 = (int)((k.n1 + bn - 1) / bn);
+  k.nblk = k.nb1 + (int)((k.L - k.n1 + bn - 1) / bn);
   return t;
 }
 

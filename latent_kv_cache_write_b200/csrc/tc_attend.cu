@@ -52,39 +52,45 @@ namespace {
 using namespace tc;
 using namespace attn;
 
-constexpr int BOX_BYTES = BN * 64 * 2;                // 64 keys x 64 dims, 8 KB
-constexpr int LAT_BYTES = 4 * BOX_BYTES;              // 32 KB of latent per stage
-constexpr int RBOX_BYTES = BN * 32 * 2;               // 64 keys x 32 RoPE dims, 4 KB
-constexpr int STAGE_BYTES = LAT_BYTES + RBOX_BYTES;   // bytes one stage's loads bring
-constexpr int QR_BYTES = TM * 32 * 2;                 // this CTA's Q RoPE part, 8 KB
-// Exchange buffer of a warpgroup, 16 KB: the peer's partial scores as fp16, chunk-major
-// [8 x 16 B][128 rows].  P buffer of a warpgroup, 16 KB: bf16, 128-byte swizzled rows.
-constexpr int XP_BYTES = TM * BN * 2;
 constexpr int NTHREADS = 352;
 
-// Shared-memory layout and barriers of the two pipeline depths.
-//   DEEP = false: 4 K/V stages; separate exchange and P buffers; an exchange buffer is
-//                 handed back to the peer as soon as its scores are read.
-//   DEEP = true:  5 K/V stages; P overwrites the exchange buffer once the scores are
-//                 read, and the PV product's commit, multicast to the peer, hands the
-//                 buffer back (the send of a block then waits for the peer's PV two
-//                 blocks earlier).  The deeper ring hides longer load latencies.
+// Three variants of one kernel, chosen per call by the host.
+//   V = 0: d_R = 64, 4 K/V stages, separate exchange and P buffers; a warpgroup hands its
+//          exchange buffer back to the peer as soon as it has read it.
+//   V = 1: d_R = 64, 5 K/V stages; P is written over the exchange buffer once the scores
+//          are read, and the PV product's commit, multicast to the peer, hands the
+//          buffer back (the send of a block then waits for the peer's PV two blocks
+//          earlier).  The deeper ring hides longer load latencies.
+//   V = 2: d_R = 512 (the wide positional key): 32-key blocks, each CTA's 256 RoPE dims
+//          as four 64-dim boxes, Q's RoPE half (64 KB) in shared memory, merged
+//          exchange/P buffers with P in 64-byte swizzled rows, 4 stages.
 // K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
-// swizzle) of stage s at OFF_KV + (q * NST + s) * BOX_BYTES, RoPE box of stage s (64-byte
-// swizzle) at OFF_KVR + s * RBOX_BYTES.
+// swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of stage s at
+// OFF_KVR + (q * NST + s) * RBB.
 // A per-block barrier completes once per use of its buffer, a per-segment one once per
 // segment; a waiter counts the uses and waits on the parity of the count.
-template <bool DEEP>
+template <int V>
 struct Lay {
-  static constexpr int NST = DEEP ? 5 : 4;
-  static constexpr bool MERGED = DEEP;
+  static constexpr bool WIDE = V == 2;
+  static constexpr int NST = V == 1 ? 5 : 4;
+  static constexpr bool MERGED = V != 0;
+  static constexpr int BNK = WIDE ? 32 : 64;                 // keys per block
+  static constexpr int BOXB = BNK * 64 * 2;                  // latent box: BNK keys x 64 dims
+  static constexpr int LATB = 4 * BOXB;                      // this CTA's latent half
+  static constexpr int NRB = WIDE ? 4 : 1;                   // RoPE boxes per stage
+  static constexpr int RDIMS = WIDE ? 64 : 32;               // dims per RoPE box
+  static constexpr int RBB = BNK * RDIMS * 2;                // RoPE box bytes
+  static constexpr int STAGEB = LATB + NRB * RBB;            // bytes one stage's loads bring
+  static constexpr int RHALF = NRB * RDIMS;                  // RoPE dims per CTA
+  static constexpr int QRB = TM * RHALF * 2;                 // this CTA's Q RoPE part
+  static constexpr int XPB = TM * BNK * 2;                   // exchange / P buffer
   static constexpr int OFF_KV = 0;
-  static constexpr int OFF_KVR = OFF_KV + NST * LAT_BYTES;
-  static constexpr int OFF_QR = OFF_KVR + NST * RBOX_BYTES;
-  static constexpr int OFF_X = OFF_QR + QR_BYTES;                 // [2] exchange buffers
-  static constexpr int OFF_P = MERGED ? OFF_X : OFF_X + 2 * XP_BYTES;   // [2] P buffers
-  static constexpr int OFF_M = OFF_P + 2 * XP_BYTES;              // running max [2][128]
-  static constexpr int OFF_L = OFF_M + 2 * TM * 4;                // final (l, m) [2][2][128]
+  static constexpr int OFF_KVR = OFF_KV + NST * LATB;
+  static constexpr int OFF_QR = OFF_KVR + NST * NRB * RBB;
+  static constexpr int OFF_X = OFF_QR + QRB;                 // [2] exchange buffers
+  static constexpr int OFF_P = MERGED ? OFF_X : OFF_X + 2 * XPB;   // [2] P buffers
+  static constexpr int OFF_M = OFF_P + 2 * XPB;              // running max [2][128]
+  static constexpr int OFF_L = OFF_M + 2 * TM * 4;           // final (l, m) [2][2][128]
   static constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
   static constexpr int B_KVF = 0;               // K/V stage loaded (TMA)                [NST]
   static constexpr int B_KVE = B_KVF + NST;     // K/V stage free (MMA commit after PV) [NST]
@@ -142,7 +148,7 @@ struct SegWalk {
   __device__ bool valid() const { return tile < tend || (tile == tend && jb < bend); }
   __device__ void load(const AttnArgs& a) {
     if (!valid()) return;
-    tg = tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, tile);
+    tg = tile_geo(a.g, a.n_q, a.q_first, a.k_first, a.n_keys, a.tiles_per_batch, tile, a.bn);
     je = tile == tend ? bend : tg.blk.nblk;
   }
   __device__ int nb() const { return je - jb; }
@@ -198,13 +204,15 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, uint32_t tq, int64_t g
   tmem_wait_st();
 }
 
-template <bool DEEP>
+template <int V>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
                   const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ AttnArgs a,
                   const __grid_constant__ Sched sc) {
-  using LY = Lay<DEEP>;
+  using LY = Lay<V>;
   constexpr int NST = LY::NST;
+  constexpr int BN = LY::BNK, BOX_BYTES = LY::BOXB, RBOX_BYTES = LY::RBB;
+  constexpr int STAGE_BYTES = LY::STAGEB, QR_BYTES = LY::QRB, XP_BYTES = LY::XPB;
   constexpr int OFF_KV = LY::OFF_KV, OFF_KVR = LY::OFF_KVR, OFF_QR = LY::OFF_QR;
   constexpr int OFF_X = LY::OFF_X, OFF_P = LY::OFF_P, OFF_M = LY::OFF_M, OFF_L = LY::OFF_L;
   constexpr int B_KVF = LY::B_KVF, B_KVE = LY::B_KVE, B_QR = LY::B_QR, B_QREADY = LY::B_QREADY;
@@ -277,8 +285,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           for (int q = 0; q < 4; ++q)
             tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
                         (int)rank * HALF + q * 64, (int32_t)slot0, sw.tg.b);
-          tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s],
-                      G.Dc + (int)rank * 32, (int32_t)slot0, sw.tg.b);
+          if constexpr (LY::WIDE) {
+#pragma unroll
+            for (int q = 0; q < LY::NRB; ++q)
+              tma_load_3d(sm + OFF_KVR + (q * NST + s) * RBOX_BYTES, &tmK, &bar[B_KVF + s],
+                          G.Dc + (int)rank * LY::RHALF + q * 64, (int32_t)slot0, sw.tg.b);
+          } else {
+            tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s],
+                        G.Dc + (int)rank * LY::RHALF, (int32_t)slot0, sw.tg.b);
+          }
         }
       }
     }
@@ -302,10 +317,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int kk = 1; kk < HALF / 16; ++kk)
           mma_ts(d, tmem + Q_COL + kk * 8,
                  kd + (uint64_t)(((kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32) >> 4), id, 1u);
-        const uint64_t qd = desc_sw64(smem_u32(sm + OFF_QR), 512);
-        const uint64_t rd = desc_sw64(smem_u32(sm + OFF_KVR + s * RBOX_BYTES), 512);
-        mma_ss(d, qd, rd, id, 1u);
-        mma_ss(d, qd + 2, rd + 2, id, 1u);              // second 16-dim step: +32 bytes
+        if constexpr (LY::WIDE) {
+          // 256 RoPE dims: Q's from its four 128-row boxes, K's from the stage's four boxes
+#pragma unroll
+          for (int kr = 0; kr < LY::RHALF / 16; ++kr) {
+            const int q = kr >> 2;
+            const uint64_t qd = desc_sw128(smem_u32(sm + OFF_QR + q * (TM * 128)) + (kr & 3) * 32,
+                                           16, 1024);
+            const uint64_t rd =
+                desc_sw128(smem_u32(sm + OFF_KVR + (q * NST + s) * RBOX_BYTES) + (kr & 3) * 32,
+                           16, 1024);
+            mma_ss(d, qd, rd, id, 1u);
+          }
+        } else {
+          const uint64_t qd = desc_sw64(smem_u32(sm + OFF_QR), 512);
+          const uint64_t rd = desc_sw64(smem_u32(sm + OFF_KVR + s * RBOX_BYTES), 512);
+          mma_ss(d, qd, rd, id, 1u);
+          mma_ss(d, qd + 2, rd + 2, id, 1u);            // second 16-dim step: +32 bytes
+        }
       };
       bool ok = true;
       for (; ok && sw.valid(); sw.next(a)) {
@@ -313,8 +342,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (sw.k > 0) ok = mbar_wait(&bar[B_QKDONE], kph ^ 1, abort, a.err, 0x107, sw.k);
         if (!ok) break;
         mbar_expect_tx(&bar[B_QR], QR_BYTES);
-        tma_load_2d(sm + OFF_QR, &tmQR, &bar[B_QR], G.Dc + (int)rank * 32,
-                    (int32_t)sw.tg.grow0);
+        if constexpr (LY::WIDE) {
+#pragma unroll
+          for (int q = 0; q < LY::NRB; ++q)
+            tma_load_2d(sm + OFF_QR + q * (TM * 128), &tmQR, &bar[B_QR],
+                        G.Dc + (int)rank * LY::RHALF + q * 64, (int32_t)sw.tg.grow0);
+        } else {
+          tma_load_2d(sm + OFF_QR, &tmQR, &bar[B_QR], G.Dc + (int)rank * LY::RHALF,
+                      (int32_t)sw.tg.grow0);
+        }
         ok = mbar_wait(&bar[B_QREADY], kph, abort, a.err, 0x102, sw.k);
         if (ok) ok = mbar_wait(&bar[B_QR], kph, abort, a.err, 0x103, sw.k);
         if (!ok) break;
@@ -358,10 +394,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const uint32_t v0 = smem_u32(sm + OFF_KV + s * BOX_BYTES);
           const uint32_t pa = smem_u32(sm + OFF_P + pb * XP_BYTES);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
-                   desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            // P is K-major: 128-byte swizzled rows of 64 keys, or 64-byte rows of 32
+            const uint64_t pd = LY::WIDE ? desc_sw64(pa + ks * 32, 512)
+                                         : desc_sw128(pa + ks * 32, 16, 1024);
+            mma_ss(tmem + O_COL, pd, desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
                    (jl > 0 || ks > 0) ? 1u : 0u);
+          }
           mma_commit(&bar[B_PE + pb]);
           mma_commit(&bar[B_KVE + s]);
           if constexpr (LY::MERGED) mma_commit_cluster(&bar[B_XE + pb], (uint16_t)(1u << peer));
@@ -380,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
     const uint32_t peer_xe = mapa(smem_u32(&bar[B_XE + wg]), peer);
     const uint4* my_x = reinterpret_cast<const uint4*>(sm + OFF_X + wg * XP_BYTES) + t;
-    uint8_t* prow = sm + OFF_P + wg * XP_BYTES + t * 128;    // P row t
+    uint8_t* prow = sm + OFF_P + wg * XP_BYTES + t * (BN * 2);   // P row t
     const float c2 = a.scale_log2;
     bool ok = true;
 
@@ -423,17 +462,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           break;
         }
         tc_fence_after();
-        float s[64];
+        float s[BN];
         {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tmem + lane_base + S_COL + wg * BN, v0);
-          tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v1);
+          uint32_t v[BN / 32][32];
+#pragma unroll
+          for (int h = 0; h < BN / 32; ++h) tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32 * h, v[h]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            s[c] = __uint_as_float(v0[c]);
-            s[32 + c] = __uint_as_float(v1[c]);
-          }
+          for (int h = 0; h < BN / 32; ++h)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) s[32 * h + c] = __uint_as_float(v[h][c]);
         }
         tc_fence_before();
         mbar_arrive(&bar[B_SE + wg]);
@@ -447,14 +485,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           break;
         }
         // the peer receives this partial rounded to fp16 (~2^-11 of a partial score)
-        uint32_t hs[32];
+        uint32_t hs[BN / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < BN / 2; ++c) {
           __half2 h2 = __floats2half2_rn(s[2 * c], s[2 * c + 1]);
           hs[c] = *reinterpret_cast<uint32_t*>(&h2);
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+        for (int q = 0; q < BN / 8; ++q)
           st_async_v4(peer_x + q * (TM * 16), hs[4 * q], hs[4 * q + 1], hs[4 * q + 2],
                       hs[4 * q + 3], peer_xf);
 
@@ -481,7 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           break;
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < BN / 8; ++q) {
           const uint4 x = my_x[q * TM];
           const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -501,11 +539,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int lim = lim64 < valid ? (lim64 < 0 ? 0 : (int)lim64) : valid;
         if (lim < BN) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+          for (int c = 0; c < BN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
         float rmax = s[0];
 #pragma unroll
-        for (int c = 1; c < 64; ++c) rmax = fmaxf(rmax, s[c]);
+        for (int c = 1; c < BN; ++c) rmax = fmaxf(rmax, s[c]);
         const float mb = rmax * c2;
 
         // running maximum after the previous block (published by the other warpgroup)
@@ -530,10 +568,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&bar[B_M + wg]);
 
         const float msub = m == -INFINITY ? 0.f : m;
-        uint32_t pk[32];
+        uint32_t pk[BN / 2];
         float sum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < BN / 2; ++c) {
           const float p0 = ex2(fmaf(s[2 * c], c2, -msub));
           const float p1 = ex2(fmaf(s[2 * c + 1], c2, -msub));
           sum += p0 + p1;
@@ -561,10 +599,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             break;
           }
         }
+        // P row t, 16-byte chunks in the hardware swizzle of its row width (128-byte
+        // rows: chunk ^ (row & 7); 64-byte rows: chunk ^ ((row >> 1) & 3))
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
+        for (int c = 0; c < BN / 8; ++c) {
+          const int cs = LY::WIDE ? (c ^ ((t >> 1) & 3)) : (c ^ (t & 7));
+          *reinterpret_cast<uint4*>(prow + cs * 16) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar[B_PF + wg]);
@@ -672,21 +714,29 @@ int cluster_slots() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (dev < 64 && cached[dev] > 0) return cached[dev];
-  if (cudaFuncSetAttribute(attend_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Lay<false>::SMEM) != cudaSuccess ||
-      cudaFuncSetAttribute(attend_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Lay<true>::SMEM) != cudaSuccess)
-    return 0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * MAXC);
-  cfg.blockDim = dim3(NTHREADS);
-  int n = 0, n2 = 0;
-  cfg.dynamicSmemBytes = Lay<false>::SMEM;
-  cudaError_t e1 = cudaOccupancyMaxActiveClusters(&n, attend_kernel<false>, &cfg);
-  cfg.dynamicSmemBytes = Lay<true>::SMEM;
-  cudaError_t e2 = cudaOccupancyMaxActiveClusters(&n2, attend_kernel<true>, &cfg);
-  if (e1 == cudaSuccess && e2 == cudaSuccess) n = n < n2 ? n : n2;
-  if (e1 != cudaSuccess || e2 != cudaSuccess || n < 1) {
+  // every variant is resident at one CTA per SM; the schedule (and the workspace size)
+  // uses the smallest count any of them reaches
+  int n = MAXC;
+  bool ok = true;
+  auto probe = [&](auto kern, int smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess) {
+      ok = false;
+      return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * MAXC);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) != cudaSuccess || c < 1) c = 0;
+    n = c < n ? c : n;
+  };
+  probe(attend_kernel<0>, Lay<0>::SMEM);
+  probe(attend_kernel<1>, Lay<1>::SMEM);
+  probe(attend_kernel<2>, Lay<2>::SMEM);
+  if (!ok) return 0;
+  if (n < 1) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return 0;
@@ -701,7 +751,9 @@ size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc + 2) * sizeo
 
 }  // namespace
 
-bool tc_attend_supported(const Geo& g) { return g.Dc == 2 * HALF && g.Dr == 64; }
+bool tc_attend_supported(const Geo& g) {
+  return g.Dc == 2 * HALF && (g.Dr == 2 * Lay<0>::RHALF || g.Dr == 2 * Lay<2>::RHALF);
+}
 
 size_t tc_attend_workspace(const Geo& g) { return 2 * (size_t)cluster_slots() * slot_bytes(g); }
 
@@ -710,20 +762,30 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
                       const void* cache, int64_t k_first, int64_t n_keys, float scale,
                       void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
                       unsigned int* err, cudaStream_t st) {
+  // variant: the wide positional key, else by whether tiles share their keys (a tile
+  // whose keys no other tile reads streams them from HBM, where the deeper ring hides the
+  // latency; keys shared by many tiles mostly hit in L2, where the shorter hand-back of
+  // the exchange buffer matters more: both measured on the video-chunk and decode shapes)
+  const int tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
+  const int variant = g.Dr == 2 * Lay<2>::RHALF ? 2 : (tiles_per_batch <= 2 ? 1 : 0);
+  const int bn = variant == 2 ? Lay<2>::BNK : Lay<0>::BNK;
   CUtensorMap K, KR, QR;
   {
+    // K: 64-dim boxes of bn cached rows (the latent boxes, and the wide RoPE boxes);
+    // KR: the 32-dim RoPE box of d_R = 64 (64-byte swizzle)
     uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.S, (uint64_t)g.B};
     uint64_t s[2] = {(uint64_t)g.row * 2, (uint64_t)g.S * g.row * 2};
-    uint32_t b[3] = {64, BN, 1};
+    uint32_t b[3] = {64, (uint32_t)bn, 1};
     if (!make_tmap_bf16(&K, cache, 3, d, s, b)) return cudaErrorInvalidValue;
-    uint32_t br[3] = {32, BN, 1};
+    uint32_t br[3] = {32, (uint32_t)bn, 1};
     if (!make_tmap_bf16(&KR, cache, 3, d, s, br, true)) return cudaErrorInvalidValue;
   }
   {
+    // Q's RoPE part: one 32-dim box (64-byte swizzle), or 64-dim boxes (wide)
     uint64_t d[2] = {(uint64_t)g.row, (uint64_t)g.B * n_q * g.H};
     uint64_t s[1] = {(uint64_t)g.row * 2};
-    uint32_t b[2] = {32, TM};
-    if (!make_tmap_bf16(&QR, q_abs, 2, d, s, b, true)) return cudaErrorInvalidValue;
+    uint32_t b[2] = {variant == 2 ? 64u : 32u, TM};
+    if (!make_tmap_bf16(&QR, q_abs, 2, d, s, b, variant != 2)) return cudaErrorInvalidValue;
   }
   const int ncl = cluster_slots();
   if (ncl == 0) return cudaErrorInvalidDevice;
@@ -734,7 +796,8 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.q_abs = (const bf16*)q_abs;
   a.o_lat = (bf16*)o_lat;
   a.lse = lse;
-  a.tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
+  a.tiles_per_batch = tiles_per_batch;
+  a.bn = bn;
   a.err = err;
   const int T = g.B * a.tiles_per_batch;
 
@@ -743,7 +806,7 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   std::vector<int64_t> pre(T + 1, 0);
   std::vector<int> nbt(T);
   for (int t = 0; t < T; ++t) {
-    nbt[t] = tile_geo(g, n_q, q_first, k_first, n_keys, a.tiles_per_batch, t).blk.nblk;
+    nbt[t] = tile_geo(g, n_q, q_first, k_first, n_keys, a.tiles_per_batch, t, bn).blk.nblk;
     pre[t + 1] = pre[t] + nbt[t];
   }
   const int64_t W = pre[T];
@@ -832,14 +895,12 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   }
   if (G == 0) return cudaSuccess;
 
-  // A tile whose keys no other tile reads streams them from HBM: the deeper ring hides
-  // that latency.  Keys shared by many tiles mostly hit in L2, where the shorter
-  // hand-back of the exchange buffer matters more (both measured on the video-chunk
-  // and decode shapes).
-  if (a.tiles_per_batch <= 2)
-    attend_kernel<true><<<(unsigned)(2 * G), NTHREADS, Lay<true>::SMEM, st>>>(K, KR, QR, a, sc);
+  if (variant == 2)
+    attend_kernel<2><<<(unsigned)(2 * G), NTHREADS, Lay<2>::SMEM, st>>>(K, KR, QR, a, sc);
+  else if (variant == 1)
+    attend_kernel<1><<<(unsigned)(2 * G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, sc);
   else
-    attend_kernel<false><<<(unsigned)(2 * G), NTHREADS, Lay<false>::SMEM, st>>>(K, KR, QR, a, sc);
+    attend_kernel<0><<<(unsigned)(2 * G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, sc);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);

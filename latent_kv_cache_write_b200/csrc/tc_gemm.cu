@@ -30,11 +30,14 @@ constexpr int STG_BYTES = 32 * 64;                // per epilogue warp: 32 rows 
 constexpr int RB_BYTES = GBM * GBN * 4;          // split-K partial accumulator, 64 KB
 // Shared memory: the stage ring, barriers, the RoPE frequency table, epilogue staging and,
 // with split-K, the buffer the other CTA of the pair sends its fp32 partial tile into.
+constexpr int OBOX_BYTES = GBM * 64 * 2;         // TMA-store box: 128 rows x 64 cols bf16
 template <int ST, bool SK> struct GLay {
   static constexpr int OFF_TAB = ST * STAGE_BYTES + 256;
   static constexpr int OFF_STG = OFF_TAB + MAX_PAIRS * 8;
   static constexpr int OFF_RB = OFF_STG + 4 * STG_BYTES;
-  static constexpr int SMEM = OFF_RB + (SK ? RB_BYTES : 0) + 1024;
+  // output boxes for the TMA stores of the absorption and the up-projection [2]
+  static constexpr int OFF_OST = (OFF_RB + (SK ? RB_BYTES : 0) + 1023) & ~1023;
+  static constexpr int SMEM = OFF_OST + (SK ? 0 : 2 * OBOX_BYTES) + 1024;
 };
 
 enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
@@ -63,7 +66,8 @@ struct TcGemm {
 template <int GSTAGES, bool SPLITK>
 __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, TcGemm p) {
+                   const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmO,
+                   TcGemm p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
     // split-K partial tile, chunk-major [32 chunks of 4 floats][128 rows]: conflict-free
     // for both the sending and the reading thread of a row
     const float4* rb = reinterpret_cast<const float4*>(smem + GL::OFF_RB) + r;
-    uint32_t tc = 0;
+    uint32_t tc = 0, ost = 0;                   // ost: output boxes stored so far
     for (int t = t_first; t < ntiles; t += t_step, ++tc) {
       int m0, n0, z;
       tile_coords(t, m0, n0, z);
@@ -288,6 +292,35 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
           tc_fence_before();
           mbar_arrive(&acce[acc]);              // accumulator may be overwritten
         }
+        if (!SPLITK && p.mode != MODE_CACHE) {
+          // The absorption's and the up-projection's outputs are plain 3-D tensors: the
+          // warps fill one 128-row x 64-column box (128-byte swizzle) of a two-buffer
+          // ring and one thread stores it with TMA, which writes the rows whole.
+          uint8_t* ob = smem + GL::OFF_OST + (ost & 1) * OBOX_BYTES;
+          ++ost;
+          if (r == 0) bulk_wait_group_read<1>();   // the store that last read `ob` is done
+          named_bar(1, 128);
+          if (ok) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t* w = &v[hh][8 * q];
+                *reinterpret_cast<uint4*>(ob + r * 128 + (((4 * hh + q) ^ (r & 7)) * 16)) =
+                    make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                               pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                               pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                               pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7])));
+              }
+          }
+          fence_proxy_async_smem();
+          named_bar(1, 128);
+          if (ok && r == 0 && n0 + c0 < p.N) {
+            tma_store_3d(&tmO, ob, n0 + c0, z, m0);
+            bulk_commit_group();
+          }
+          continue;
+        }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int n = n0 + c0 + 32 * hh;      // output column of v[hh][0] (warp-uniform)
@@ -367,6 +400,8 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
       }
       if (!ok) break;
     }
+    // the output boxes' stores have finished with shared memory and landed before exit
+    if (r == 0) bulk_wait_group<0>();
   }
   __syncwarp();
   tc_fence_before();
@@ -391,7 +426,7 @@ int sm_count() {
 
 template <int ST, bool SK>
 cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
-                      const TcGemm& q, long long tiles, cudaStream_t st) {
+                      const CUtensorMap& O, const TcGemm& q, long long tiles, cudaStream_t st) {
   using GL = GLay<ST, SK>;
   {
     // the shared-memory opt-in is per device
@@ -412,7 +447,7 @@ cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
     const long long slots = (long long)sm_count() * (ST == 2 ? 2 : 1);
     const int grid = (int)(tiles < slots ? tiles : slots);
     if (grid == 0) return cudaSuccess;
-    tc_gemm_kernel<ST, SK><<<grid, GTHREADS, GL::SMEM, st>>>(A, B, B2, q);
+    tc_gemm_kernel<ST, SK><<<grid, GTHREADS, GL::SMEM, st>>>(A, B, B2, O, q);
   } else {
     // clusters of two CTAs, one cluster per tile up to one per SM pair
     const long long pairs = sm_count() / 2;
@@ -430,7 +465,7 @@ cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<ST, SK>, A, B, B2, q);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<ST, SK>, A, B, B2, O, q);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = cudaGetLastError();
@@ -439,18 +474,18 @@ cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
 }
 
 cudaError_t launch(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
-                   const TcGemm& p, int zcount, cudaStream_t st) {
+                   const CUtensorMap& O, const TcGemm& p, int zcount, cudaStream_t st) {
   TcGemm q = p;
   q.Z = zcount;
   const long long tiles =
       (long long)((p.M + GBM - 1) / GBM) * ((p.N + GBN - 1) / GBN) * zcount;
   const int nk = (p.K + GBK - 1) / GBK;
   // the absorption's tiles are two K-blocks long: two CTAs per SM hide their latency
-  if (p.mode == MODE_ABSORB) return launch_st<2, false>(A, B, B2, q, tiles, st);
+  if (p.mode == MODE_ABSORB) return launch_st<2, false>(A, B, B2, O, q, tiles, st);
   // fewer tiles than SMs and a long K loop (the cache write): split K over CTA pairs
   if (p.mode == MODE_CACHE && nk >= 2 && tiles < sm_count())
-    return launch_st<4, true>(A, B, B2, q, tiles, st);
-  return launch_st<4, false>(A, B, B2, q, tiles, st);
+    return launch_st<4, true>(A, B, B2, O, q, tiles, st);
+  return launch_st<4, false>(A, B, B2, O, q, tiles, st);
 }
 
 }  // namespace
@@ -490,7 +525,7 @@ cudaError_t tc_cache_write(const Geo& g, const void* h, int d_model, int64_t n_t
   p.M = (int)rows; p.N = g.row; p.K = d_model; p.mode = MODE_CACHE; p.b_mn = 1;
   p.n_split = g.Dc; p.out = (bf16*)cache; p.rows_per_batch = n_tok; p.geo = g;
   p.first_tok = first_tok; p.slots = slots; p.err = err;
-  return launch(A, B, B2, p, 1, st);
+  return launch(A, B, B2, B, p, 1, st);       // the cache write stores without TMA
 }
 
 cudaError_t tc_absorb_q(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,
@@ -514,7 +549,15 @@ cudaError_t tc_absorb_q(const Geo& g, const void* q_nope, const void* q_rope, in
   p.M = (int)rows; p.N = g.Dc; p.K = g.Dn; p.mode = MODE_ABSORB; p.b_mn = 1;
   p.n_split = 1 << 30; p.out = (bf16*)q_abs; p.rows_per_batch = n_q; p.geo = g;
   p.first_tok = q_first; p.q_rope = (const bf16*)q_rope; p.err = err;
-  return launch(A, B, B, p, g.H, st);
+  CUtensorMap O;
+  {
+    // q_abs as (d_c + d_R, heads, rows): 64-column boxes of 128 rows of one head
+    uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.H, rows};
+    uint64_t s[2] = {(uint64_t)g.row * 2, (uint64_t)g.H * g.row * 2};
+    uint32_t b[3] = {64, 1, (uint32_t)GBM};
+    if (!make_tmap_bf16(&O, q_abs, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  return launch(A, B, B, O, p, g.H, st);
 }
 
 cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_uv, void* out,
@@ -536,7 +579,15 @@ cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_
   TcGemm p{};
   p.M = (int)rows; p.N = g.Dn; p.K = g.Dc; p.mode = MODE_UPV; p.b_mn = 0;
   p.n_split = 1 << 30; p.out = (bf16*)out; p.rows_per_batch = n_q; p.geo = g; p.err = err;
-  return launch(A, B, B, p, g.H, st);
+  CUtensorMap O;
+  {
+    // out as (d_nope, heads, rows): 64-column boxes of 128 rows of one head
+    uint64_t d[3] = {(uint64_t)g.Dn, (uint64_t)g.H, rows};
+    uint64_t s[2] = {(uint64_t)g.Dn * 2, (uint64_t)g.H * g.Dn * 2};
+    uint32_t b[3] = {64, 1, (uint32_t)GBM};
+    if (!make_tmap_bf16(&O, out, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  return launch(A, B, B, O, p, g.H, st);
 }
 
 }  // namespace mla

@@ -64,15 +64,6 @@ __device__ __forceinline__ void rope_rotate(float& a, float& b, double ang) {
   b = (float)nb;
 }
 
-// Axis position of token g for RoPE pair p, and the pair's frequency theta^(-j/n).
-__device__ __forceinline__ int64_t rope_pos(const Geo& G, int64_t g, int p) {
-  const int64_t t = g / G.F;
-  const int64_t r = g - t * G.F;
-  if (p < G.pairs[0]) return t;
-  const int64_t y = r / G.gw;
-  if (p < G.pairs[0] + G.pairs[1]) return y;
-  return r - y * G.gw;
-}
 // The three axis positions (t, y, x) of token g, as doubles, computed once per token;
 // rope_axis_pos picks the one RoPE pair p turns by.
 struct RopeAxes {
@@ -87,6 +78,7 @@ __device__ __forceinline__ RopeAxes rope_axes(const Geo& G, int64_t g) {
 __device__ __forceinline__ double rope_axis_pos(const Geo& G, const RopeAxes& ax, int p) {
   return p < G.pairs[0] ? ax.t : (p < G.pairs[0] + G.pairs[1] ? ax.y : ax.x);
 }
+// The frequency theta^(-j/n) of RoPE pair p (pair j of an axis segment with n pairs).
 __device__ __forceinline__ double rope_inv_freq(const Geo& G, int p) {
   int j, n;
   if (p < G.pairs[0]) {

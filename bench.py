@@ -355,23 +355,29 @@ def cpu_baseline(seconds: float = 12.0):
             "seconds": dt}
 
 
-# DRAM bytes (read + write) of one chunk attention launch, from the ncu capture summarised in
-# profiles/attend_kernel_video_chunk.md.  Counters describe the kernel source they were
-# taken on: the value is reported only while that source is unchanged.
-ATTEND_TRAFFIC = {"bytes": 73_488_384 + 32_379_136,
-                  "source": "latent_kv_cache_write_b200/csrc/tc_attend.cu",
-                  "sha256": "04cfb0a9b3a0f490168e311e044c6643184007c907ad195918a34e09e85b63c8"}
+# DRAM bytes (read + write) of one chunk mla_attend call, from the ncu captures summarised in
+# profiles/attend_kernel_video_chunk.md (the attention kernel) and
+# profiles/combine_kernel_video_chunk.md (the split-key merge).  Counters describe the kernel
+# sources they were taken on: the value is reported only while those sources are unchanged.
+ATTEND_TRAFFIC = {"bytes": (73_514_752 + 32_410_112) + (37_907_968 + 16_896),
+                  "sources": {
+                      "latent_kv_cache_write_b200/csrc/tc_attend.cu":
+                          "ee3ead6fdc25fce6408c5565558b278562449917720a61732bb010df7ac848dd",
+                      "latent_kv_cache_write_b200/csrc/attend_combine.cu":
+                          "67947231c23dc78cb22b69f230758b971516c21f6b7bbc699d9acefd11dc1ca6"}}
 
 
 def attend_traffic():
     import hashlib
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), ATTEND_TRAFFIC["source"])
-    try:
-        with open(path, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-    except OSError:
-        return None
-    return ATTEND_TRAFFIC["bytes"] if digest == ATTEND_TRAFFIC["sha256"] else None
+    root = os.path.dirname(os.path.abspath(__file__))
+    for rel, want in ATTEND_TRAFFIC["sources"].items():
+        try:
+            with open(os.path.join(root, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != want:
+                    return None
+        except OSError:
+            return None
+    return ATTEND_TRAFFIC["bytes"]
 
 
 def ranks_max(value: float, dist, device) -> float:

@@ -54,16 +54,14 @@ using namespace attn;
 
 constexpr int NTHREADS = 352;
 
-// Three variants of one kernel, chosen per call by the host.
-//   V = 0: d_R = 64, 4 K/V stages, separate exchange and P buffers; a warpgroup hands its
-//          exchange buffer back to the peer as soon as it has read it.
-//   V = 1: d_R = 64, 5 K/V stages; P is written over the exchange buffer once the scores
-//          are read, and the PV product's commit, multicast to the peer, hands the
-//          buffer back (the send of a block then waits for the peer's PV two blocks
-//          earlier).  The deeper ring hides longer load latencies.
-//   V = 2: d_R = 512 (the wide positional key): 32-key blocks, each CTA's 256 RoPE dims
-//          as four 64-dim boxes, Q's RoPE half (64 KB) in shared memory, merged
-//          exchange/P buffers with P in 64-byte swizzled rows, 4 stages.
+// Two variants of one kernel, chosen per call by the host.
+//   V = 0: d_R = 64: 64-key blocks, 4 K/V stages, separate exchange and P buffers; a
+//          warpgroup hands its exchange buffer back to the peer as soon as it has read it.
+//   V = 1: d_R = 512 (the wide positional key): 32-key blocks, each CTA's 256 RoPE dims
+//          as four 64-dim boxes, Q's RoPE half (64 KB) in shared memory, 4 stages.  P is
+//          written over the exchange buffer once the scores are read (8 KB each, P in
+//          64-byte swizzled rows), and the PV product's commit, multicast to the peer,
+//          hands the buffer back.
 // K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
 // swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of stage s at
 // OFF_KVR + (q * NST + s) * RBB.
@@ -71,9 +69,9 @@ constexpr int NTHREADS = 352;
 // segment; a waiter counts the uses and waits on the parity of the count.
 template <int V>
 struct Lay {
-  static constexpr bool WIDE = V == 2;
-  static constexpr int NST = V == 1 ? 5 : 4;
-  static constexpr bool MERGED = V != 0;
+  static constexpr bool WIDE = V == 1;
+  static constexpr int NST = 4;
+  static constexpr bool MERGED = WIDE;
   static constexpr int BNK = WIDE ? 32 : 64;                 // keys per block
   static constexpr int BOXB = BNK * 64 * 2;                  // latent box: BNK keys x 64 dims
   static constexpr int LATB = 4 * BOXB;                      // this CTA's latent half
@@ -734,7 +732,6 @@ int cluster_slots() {
   };
   probe(attend_kernel<0>, Lay<0>::SMEM);
   probe(attend_kernel<1>, Lay<1>::SMEM);
-  probe(attend_kernel<2>, Lay<2>::SMEM);
   if (!ok) return 0;
   if (n < 1) {
     int sms = 0;
@@ -752,7 +749,7 @@ size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc + 2) * sizeo
 }  // namespace
 
 bool tc_attend_supported(const Geo& g) {
-  return g.Dc == 2 * HALF && (g.Dr == 2 * Lay<0>::RHALF || g.Dr == 2 * Lay<2>::RHALF);
+  return g.Dc == 2 * HALF && (g.Dr == 2 * Lay<0>::RHALF || g.Dr == 2 * Lay<1>::RHALF);
 }
 
 size_t tc_attend_workspace(const Geo& g) { return 2 * (size_t)cluster_slots() * slot_bytes(g); }
@@ -762,13 +759,9 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
                       const void* cache, int64_t k_first, int64_t n_keys, float scale,
                       void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
                       unsigned int* err, cudaStream_t st) {
-  // variant: the wide positional key, else by whether tiles share their keys (a tile
-  // whose keys no other tile reads streams them from HBM, where the deeper ring hides the
-  // latency; keys shared by many tiles mostly hit in L2, where the shorter hand-back of
-  // the exchange buffer matters more: both measured on the video-chunk and decode shapes)
   const int tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
-  const int variant = g.Dr == 2 * Lay<2>::RHALF ? 2 : (tiles_per_batch <= 2 ? 1 : 0);
-  const int bn = variant == 2 ? Lay<2>::BNK : Lay<0>::BNK;
+  const int variant = g.Dr == 2 * Lay<1>::RHALF ? 1 : 0;      // the wide positional key
+  const int bn = variant == 1 ? Lay<1>::BNK : Lay<0>::BNK;
   CUtensorMap K, KR, QR;
   {
     // K: 64-dim boxes of bn cached rows (the latent boxes, and the wide RoPE boxes);
@@ -784,8 +777,8 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     // Q's RoPE part: one 32-dim box (64-byte swizzle), or 64-dim boxes (wide)
     uint64_t d[2] = {(uint64_t)g.row, (uint64_t)g.B * n_q * g.H};
     uint64_t s[1] = {(uint64_t)g.row * 2};
-    uint32_t b[2] = {variant == 2 ? 64u : 32u, TM};
-    if (!make_tmap_bf16(&QR, q_abs, 2, d, s, b, variant != 2)) return cudaErrorInvalidValue;
+    uint32_t b[2] = {variant == 1 ? 64u : 32u, TM};
+    if (!make_tmap_bf16(&QR, q_abs, 2, d, s, b, variant != 1)) return cudaErrorInvalidValue;
   }
   const int ncl = cluster_slots();
   if (ncl == 0) return cudaErrorInvalidDevice;
@@ -895,9 +888,7 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   }
   if (G == 0) return cudaSuccess;
 
-  if (variant == 2)
-    attend_kernel<2><<<(unsigned)(2 * G), NTHREADS, Lay<2>::SMEM, st>>>(K, KR, QR, a, sc);
-  else if (variant == 1)
+  if (variant == 1)
     attend_kernel<1><<<(unsigned)(2 * G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, sc);
   else
     attend_kernel<0><<<(unsigned)(2 * G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, sc);

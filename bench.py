@@ -34,7 +34,10 @@ sys.path.insert(0, ROOT)
 from synth import configs as C  # noqa: E402
 from synth import generate as G  # noqa: E402
 
-WORKLOAD = C.VIDEO_CHUNK
+WORKLOAD = C.VIDEO_CHUNK            # the default step; --workload picks another
+# workloads whose step writes its own cache (decode reads a cache given directly and is
+# timed by the decode leg)
+STEP_WORKLOADS = tuple(w.name for w in C.ALL if not w.cache_direct and w.elem_bytes == 2)
 L2_FLUSH_BYTES = 256 << 20           # > 126 MB L2: written between timed steps
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -310,12 +313,11 @@ def decode_leg(torch, mla, steps, warmup, flush):
             "tflops": step_flops(wl)["attend"] / (t * 1e-3) / 1e12}
 
 
-def cpu_baseline(seconds: float = 12.0):
+def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
     """The fp64 oracle, as it stands, on a bounded sample of the same step: the cache
     write, absorption, absorbed attention and up-projection of a prefix of the chunk's
     queries (all heads), repeated until ``seconds`` elapse."""
     import oracle.mla_oracle as O
-    wl = WORKLOAD
     w = {k: v.values for k, v in G.weights(wl, 0).items()}
     F = wl.tokens_per_frame
     rng_cache = np.zeros((wl.batch, wl.ring_slots, wl.row_width))
@@ -349,9 +351,10 @@ def cpu_baseline(seconds: float = 12.0):
     except Exception:  # noqa: BLE001
         threads = os.cpu_count()
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {n_q} of {wl.n_queries} chunk queries (all {wl.n_heads} heads, "
-                      f"{wl.n_keys} keys): cache write, absorption, latent attention, "
-                      f"up-projection in fp64 NumPy; {dt:.1f} s",
+            "sample": f"first {n_q} of {wl.n_queries} chunk queries"
+                      + (f" of each of {wl.batch} sequences" if wl.batch > 1 else "")
+                      + f" (all {wl.n_heads} heads, {wl.n_keys} keys): cache write, absorption, "
+                      f"latent attention, up-projection in fp64 NumPy; {dt:.1f} s",
             "seconds": dt}
 
 
@@ -359,16 +362,19 @@ def cpu_baseline(seconds: float = 12.0):
 # profiles/attend_kernel_video_chunk.md (the attention kernel) and
 # profiles/combine_kernel_video_chunk.md (the split-key merge).  Counters describe the kernel
 # sources they were taken on: the value is reported only while those sources are unchanged.
-ATTEND_TRAFFIC = {"bytes": (73_514_752 + 32_410_112) + (37_907_968 + 16_896),
+ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
+                  "bytes": (73_877_504 + 34_028_032) + (37_907_968 + 16_896),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
-                          "ee3ead6fdc25fce6408c5565558b278562449917720a61732bb010df7ac848dd",
+                          "209c6e02806d9eb047d09790a18b63f7e033957a9b3a4eff799a83b980ddf56d",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
                           "67947231c23dc78cb22b69f230758b971516c21f6b7bbc699d9acefd11dc1ca6"}}
 
 
-def attend_traffic():
+def attend_traffic(wl=WORKLOAD):
     import hashlib
+    if wl.name != ATTEND_TRAFFIC["workload"]:
+        return None
     root = os.path.dirname(os.path.abspath(__file__))
     for rel, want in ATTEND_TRAFFIC["sources"].items():
         try:
@@ -413,7 +419,7 @@ def run_ours(args):
         build.build()
     if world > 1:
         dist.barrier()
-    wl = WORKLOAD
+    wl = C.BY_NAME[args.workload]
     step = Step(wl, seed=rank, torch=torch, mla=mla)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     for _ in range(args.warmup):
@@ -465,12 +471,12 @@ def run_ours(args):
             "roofline": {"kernel": "mla_attend", "bound": "tensor", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "traffic": attend_traffic(), "traffic_unit": "B per launch (ncu)",
+                         "traffic": attend_traffic(wl), "traffic_unit": "B per launch (ncu)",
                          "ms_per_launch": att_ms},
             "e2e": {"value": job_throughput(world, flops_step, args.steps, e2e_total) / 1e12,
                     "pipelining": "upload and download streams overlap step i+1's inputs and "
                                   "step i-1's output with step i's compute; no L2 flush (a "
-                                  "step moves ~173 MB through HBM, more than L2)",
+                                  "step moves more bytes through HBM than L2 holds)",
                     "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(sum(v.nbytes for v in step.host.values())),
                     "d2h_bytes_per_step": int(step.out.numel() * 2),
@@ -481,7 +487,7 @@ def run_ours(args):
             "kernels_ms": kernels_ms,
         }
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline()
+            line["cpu_baseline"] = cpu_baseline(wl=wl)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -495,16 +501,16 @@ def run_reference(args):
     if rank != 0:
         return
     per_step_s = 4.0
+    wl = C.BY_NAME[args.workload]
     for _ in range(args.warmup):
-        cpu_baseline(seconds=0.5)
+        cpu_baseline(seconds=0.5, wl=wl)
     vals, secs = [], 0.0
     last = None
     for _ in range(args.steps):
-        last = cpu_baseline(seconds=per_step_s)
+        last = cpu_baseline(seconds=per_step_s, wl=wl)
         vals.append(last["value"])
         secs += last["seconds"]
     v = statistics.mean(vals)
-    wl = WORKLOAD
     line = {
         "impl": "reference",
         "metric": "absorbed MLA attention TFLOP/s (chunk) and latent-cache GB/s (decode) "
@@ -527,6 +533,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD.name, choices=STEP_WORKLOADS,
+                    help="the step's workload (default: the video chunk)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

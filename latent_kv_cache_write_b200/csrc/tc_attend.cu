@@ -54,14 +54,13 @@ using namespace attn;
 
 constexpr int NTHREADS = 352;
 
-// Two variants of one kernel, chosen per call by the host.
-//   V = 0: d_R = 64: 64-key blocks, 4 K/V stages, separate exchange and P buffers; a
-//          warpgroup hands its exchange buffer back to the peer as soon as it has read it.
-//   V = 1: d_R = 512 (the wide positional key): 32-key blocks, each CTA's 256 RoPE dims
-//          as four 64-dim boxes, Q's RoPE half (64 KB) in shared memory, 4 stages.  P is
-//          written over the exchange buffer once the scores are read (8 KB each, P in
-//          64-byte swizzled rows), and the PV product's commit, multicast to the peer,
-//          hands the buffer back.
+// Two variants of one kernel, chosen per call by the host; both take 64-key blocks.
+//   V = 0: d_R = 64: 4 K/V stages, separate exchange and P buffers; a warpgroup hands its
+//          exchange buffer back to the peer as soon as it has read it.
+//   V = 1: d_R = 512 (the wide positional key): each CTA's 256 RoPE dims as four 64-dim
+//          boxes, Q's RoPE half (64 KB) in shared memory, 2 K/V stages of 64 KB.  P is
+//          written over the exchange buffer once the scores are read, and the PV
+//          product's commit, multicast to the peer, hands the buffer back.
 // K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
 // swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of stage s at
 // OFF_KVR + (q * NST + s) * RBB.
@@ -70,9 +69,9 @@ constexpr int NTHREADS = 352;
 template <int V>
 struct Lay {
   static constexpr bool WIDE = V == 1;
-  static constexpr int NST = 4;
+  static constexpr int NST = WIDE ? 2 : 4;
   static constexpr bool MERGED = WIDE;
-  static constexpr int BNK = WIDE ? 32 : 64;                 // keys per block
+  static constexpr int BNK = 64;                             // keys per block
   static constexpr int BOXB = BNK * 64 * 2;                  // latent box: BNK keys x 64 dims
   static constexpr int LATB = 4 * BOXB;                      // this CTA's latent half
   static constexpr int NRB = WIDE ? 4 : 1;                   // RoPE boxes per stage
@@ -81,15 +80,14 @@ struct Lay {
   static constexpr int STAGEB = LATB + NRB * RBB;            // bytes one stage's loads bring
   static constexpr int RHALF = NRB * RDIMS;                  // RoPE dims per CTA
   static constexpr int QRB = TM * RHALF * 2;                 // this CTA's Q RoPE part
-  static constexpr int XPB = TM * BNK * 2;                   // exchange / P buffer
+  static constexpr int XPB = TM * BNK * 2;                   // exchange / P buffer (128-byte rows)
   static constexpr int OFF_KV = 0;
   static constexpr int OFF_KVR = OFF_KV + NST * LATB;
   static constexpr int OFF_QR = OFF_KVR + NST * NRB * RBB;
   static constexpr int OFF_X = OFF_QR + QRB;                 // [2] exchange buffers
   static constexpr int OFF_P = MERGED ? OFF_X : OFF_X + 2 * XPB;   // [2] P buffers
   static constexpr int OFF_M = OFF_P + 2 * XPB;              // running max [2][128]
-  static constexpr int OFF_L = OFF_M + 2 * TM * 4;           // final (l, m) [2][2][128]
-  static constexpr int OFF_BAR = OFF_L + 4 * TM * 4;
+  static constexpr int OFF_BAR = OFF_M + 2 * TM * 4;
   static constexpr int B_KVF = 0;               // K/V stage loaded (TMA)                [NST]
   static constexpr int B_KVE = B_KVF + NST;     // K/V stage free (MMA commit after PV) [NST]
   static constexpr int B_QR = B_KVE + NST;      // Q RoPE tile of a segment loaded (TMA)
@@ -104,7 +102,9 @@ struct Lay {
   static constexpr int B_PF = B_XE + 2;         // P complete, O rescaled (128)          [2]
   static constexpr int B_PE = B_PF + 2;         // PV done (MMA commit)                  [2]
   static constexpr int B_M = B_PE + 2;          // running max of a block published (128) [2]
-  static constexpr int NBAR = B_M + 2;
+  static constexpr int B_KRE = B_M + 2;         // RoPE boxes of a stage free (wide; MMA commit
+                                                // after the scores)                      [NST]
+  static constexpr int NBAR = B_KRE + NST;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
@@ -212,11 +212,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   constexpr int BN = LY::BNK, BOX_BYTES = LY::BOXB, RBOX_BYTES = LY::RBB;
   constexpr int STAGE_BYTES = LY::STAGEB, QR_BYTES = LY::QRB, XP_BYTES = LY::XPB;
   constexpr int OFF_KV = LY::OFF_KV, OFF_KVR = LY::OFF_KVR, OFF_QR = LY::OFF_QR;
-  constexpr int OFF_X = LY::OFF_X, OFF_P = LY::OFF_P, OFF_M = LY::OFF_M, OFF_L = LY::OFF_L;
+  constexpr int OFF_X = LY::OFF_X, OFF_P = LY::OFF_P, OFF_M = LY::OFF_M;
   constexpr int B_KVF = LY::B_KVF, B_KVE = LY::B_KVE, B_QR = LY::B_QR, B_QREADY = LY::B_QREADY;
   constexpr int B_QKDONE = LY::B_QKDONE, B_SEGDONE = LY::B_SEGDONE, B_OFREE = LY::B_OFREE;
   constexpr int B_SF = LY::B_SF, B_SE = LY::B_SE, B_XF = LY::B_XF, B_XE = LY::B_XE;
-  constexpr int B_PF = LY::B_PF, B_PE = LY::B_PE, B_M = LY::B_M;
+  constexpr int B_PF = LY::B_PF, B_PE = LY::B_PE, B_M = LY::B_M, B_KRE = LY::B_KRE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -233,6 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar[B_KVF + s], 1);
       mbar_init(&bar[B_KVE + s], 1);
+      mbar_init(&bar[B_KRE + s], 1);
     }
     mbar_init(&bar[B_QR], 1);
     mbar_init(&bar[B_QREADY], 256);
@@ -273,36 +274,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int j = sw.jb; j < sw.je; ++j) {
           const int g = sw.gbase + (j - sw.jb);
           const int s = g % NST;
-          ok = mbar_wait(&bar[B_KVE + s], ((g / NST) & 1) ^ 1, abort, a.err, 0x101, g);
-          if (!ok) break;
+          const uint32_t fph = ((g / NST) & 1) ^ 1;
           int64_t slot0, g0;
           int valid;
           sw.tg.blk.get(j, slot0, g0, valid);
-          mbar_expect_tx(&bar[B_KVF + s], STAGE_BYTES);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
-                        (int)rank * HALF + q * 64, (int32_t)slot0, sw.tg.b);
           if constexpr (LY::WIDE) {
+            // half of a wide stage is RoPE, read only by the score MMAs: it is refilled as
+            // soon as they are done, while the latent half waits for the PV product
+            ok = mbar_wait(&bar[B_KRE + s], fph, abort, a.err, 0x109, g);
+            if (!ok) break;
+            mbar_expect_tx(&bar[B_KVF + s], STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < LY::NRB; ++q)
               tma_load_3d(sm + OFF_KVR + (q * NST + s) * RBOX_BYTES, &tmK, &bar[B_KVF + s],
                           G.Dc + (int)rank * LY::RHALF + q * 64, (int32_t)slot0, sw.tg.b);
-          } else {
+          }
+          ok = mbar_wait(&bar[B_KVE + s], fph, abort, a.err, 0x101, g);
+          if (!ok) break;
+          if constexpr (!LY::WIDE) mbar_expect_tx(&bar[B_KVF + s], STAGE_BYTES);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
+                        (int)rank * HALF + q * 64, (int32_t)slot0, sw.tg.b);
+          if constexpr (!LY::WIDE)
             tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s],
                         G.Dc + (int)rank * LY::RHALF, (int32_t)slot0, sw.tg.b);
-          }
         }
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ score MMA issuer
-    // Scores of blocks 2i and 2i+1 of a segment are one N=128 series (S buffers 0 and 1
-    // are adjacent) when their stages are adjacent, else two N=64 series; a series is
-    // issued as soon as its data and S buffers are ready: the scores start the softmax
-    // chains.  An MMA issue blocks while the tensor pipe is busy, so the PV products
-    // have their own issuing thread.  A segment's Q RoPE tile is loaded once every score
-    // MMA of the previous segment has finished.
+    // The scores of a block are one N=64 series into the S buffer of the warpgroup that
+    // takes it, issued as soon as the block's stage has landed and the buffer has been
+    // read: the scores start the softmax chains.  An MMA issue blocks while the tensor
+    // pipe is busy, so the PV products have their own issuing thread.  A segment's Q RoPE
+    // tile is loaded once every score MMA of the previous segment has finished.
     if (lane == 0) {
       prefetch_tmap(&tmQR);
       const uint32_t id_qk1 = idesc_bf16(128, BN, false, false);
@@ -364,6 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           tc_fence_after();
           qk_series(tmem + S_COL + w * BN, s, id_qk1);
           mma_commit(&bar[B_SF + w]);
+          if constexpr (LY::WIDE) mma_commit(&bar[B_KRE + s]);
         }
         mma_commit(&bar[B_QKDONE]);
       }
@@ -393,10 +400,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const uint32_t pa = smem_u32(sm + OFF_P + pb * XP_BYTES);
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
-            // P is K-major: 128-byte swizzled rows of 64 keys, or 64-byte rows of 32
-            const uint64_t pd = LY::WIDE ? desc_sw64(pa + ks * 32, 512)
-                                         : desc_sw128(pa + ks * 32, 16, 1024);
-            mma_ss(tmem + O_COL, pd, desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
+            // P is K-major: 128-byte swizzled rows of 64 keys
+            mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
+                   desc_sw128(v0 + ks * 2048, NST * BOX_BYTES, 1024), id_pv,
                    (jl > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(&bar[B_PE + pb]);
@@ -412,7 +418,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int t = tid & (TM - 1);              // row of the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     float* m_sh = reinterpret_cast<float*>(sm + OFF_M);
-    float* l_sh = reinterpret_cast<float*>(sm + OFF_L);
     const uint32_t peer_x = mapa(smem_u32(sm + OFF_X + wg * XP_BYTES), peer) + (uint32_t)t * 16;
     const uint32_t peer_xf = mapa(smem_u32(&bar[B_XF + wg]), peer);
     const uint32_t peer_xe = mapa(smem_u32(&bar[B_XE + wg]), peer);
@@ -597,11 +602,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             break;
           }
         }
-        // P row t, 16-byte chunks in the hardware swizzle of its row width (128-byte
-        // rows: chunk ^ (row & 7); 64-byte rows: chunk ^ ((row >> 1) & 3))
+        // P row t, 16-byte chunks in the 128-byte hardware swizzle (chunk ^ (row & 7))
 #pragma unroll
         for (int c = 0; c < BN / 8; ++c) {
-          const int cs = LY::WIDE ? (c ^ ((t >> 1) & 3)) : (c ^ (t & 7));
+          const int cs = c ^ (t & 7);
           *reinterpret_cast<uint4*>(prow + cs * 16) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
@@ -629,14 +633,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // ---------------------------------------------------------- segment epilogue
       if (!__all_sync(FULL, mbar_wait(&bar[B_SEGDONE], kph, abort, a.err, 0x401, t))) break;
       tc_fence_after();
-      l_sh[(wg * 2) * TM + t] = l;
-      l_sh[(wg * 2 + 1) * TM + t] = m_last;
+      // the two warpgroups' (l, m) meet in the running-max array, which no block of this
+      // segment reads any more (a warpgroup that gets here first rewrites its slot with
+      // the value it published last): the maxima, then the sums at the common maximum
+      m_sh[wg * TM + t] = m_last;
       named_bar(3, 2 * TM);
-      const float l0 = l_sh[t], m0 = l_sh[TM + t], l1 = l_sh[2 * TM + t], m1 = l_sh[3 * TM + t];
-      named_bar(3, 2 * TM);                  // both warpgroups have read (l, m)
-      const float mf = fmaxf(m0, m1);
-      const float lt = (m0 > -INFINITY ? l0 * ex2(m0 - mf) : 0.f) +
-                       (m1 > -INFINITY ? l1 * ex2(m1 - mf) : 0.f);
+      const float mf = fmaxf(m_last, m_sh[(wg ^ 1) * TM + t]);
+      named_bar(3, 2 * TM);
+      m_sh[wg * TM + t] = m_last > -INFINITY ? l * ex2(m_last - mf) : 0.f;
+      named_bar(3, 2 * TM);
+      const float lt = m_sh[t] + m_sh[TM + t];
+      named_bar(3, 2 * TM);                  // both have read: the array is the next segment's
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const float lse_v = lt > 0.f ? (mf + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
       const bool part = sw.partial();
@@ -792,113 +799,143 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.tiles_per_batch = tiles_per_batch;
   a.bn = bn;
   a.err = err;
-  const int T = g.B * a.tiles_per_batch;
-
-  // ---- schedule: the blocks of all tiles end to end, one equal range per cluster
   const bool split = workspace != nullptr && workspace_bytes >= tc_attend_workspace(g);
-  std::vector<int64_t> pre(T + 1, 0);
-  std::vector<int> nbt(T);
-  for (int t = 0; t < T; ++t) {
-    nbt[t] = tile_geo(g, n_q, q_first, k_first, n_keys, a.tiles_per_batch, t, bn).blk.nblk;
-    pre[t + 1] = pre[t] + nbt[t];
-  }
-  const int64_t W = pre[T];
-  // Two candidate schedules, costed in key blocks: a cluster's blocks plus SEG_COST per
-  // segment it walks (the switch: Q reload, output epilogue, pipeline refill), plus
-  // COMBINE_COST when tiles are split (the merge launch).  Both costs were measured on
-  // B200 (video chunk, long window and decode shapes).
-  constexpr int64_t SEG_COST = 7, COMBINE_COST = 16;
-  auto cost = [&](const Sched& c, int nc) {
-    int64_t worst = 0;
-    bool any_split = false;
-    for (int k = 0; k < nc; ++k) {
-      const int t0 = c.cut_tile[k], b0 = c.cut_blk[k], t1 = c.cut_tile[k + 1], b1 = c.cut_blk[k + 1];
-      const int64_t blocks = (pre[t1] + b1) - (pre[t0] + b0);
-      const int64_t segs = (int64_t)(t1 - t0) + (b1 > 0 ? 1 : 0);
-      any_split = any_split || b0 > 0 || b1 > 0;
-      worst = blocks + SEG_COST * segs > worst ? blocks + SEG_COST * segs : worst;
-    }
-    return worst + (any_split ? COMBINE_COST : 0);
-  };
-  // cuts on tile boundaries: the first one at or past an equal share of the blocks (of the
-  // tiles when there are no blocks)
-  Sched whole{};
-  const int G_whole = T < ncl ? T : ncl;
-  {
-    int t = 0;
-    for (int c = 1; c <= G_whole; ++c) {
-      if (c == G_whole) {
-        t = T;
-      } else if (W > 0) {
-        const int64_t pos = W * c / G_whole;
-        while (t < T && pre[t] < pos) ++t;
-      } else {
-        t = (int)((int64_t)T * c / G_whole);
-      }
-      whole.cut_tile[c] = t;
-      whole.cut_blk[c] = 0;
-    }
-  }
-  Sched sc = whole;
-  int G = G_whole;
-  if (split && W > 0) {
-    // cut c at block W*c/G; tiles without blocks go with the range before them
-    Sched sk{};
-    const int G_split = (int)(W < ncl ? W : ncl);
-    int t = 0;
-    for (int c = 1; c <= G_split; ++c) {
-      const int64_t pos = W * c / G_split;
-      while (t < T && pre[t + 1] <= pos) ++t;      // tile holding block `pos`
-      sk.cut_tile[c] = t;
-      sk.cut_blk[c] = t < T ? (int)(pos - pre[t]) : 0;
-    }
-    if (cost(sk, G_split) < cost(whole, G_whole)) {
-      sc = sk;
-      G = G_split;
-    }
-  }
-  sc.cut_tile[0] = 0;
-  sc.cut_blk[0] = 0;
-  // partial segments: their workspace slots, and the tiles to combine
-  CombineList cl{};
-  int nslot = 0;
-  for (int c = 0; c < G; ++c) {
-    sc.slot0[c] = nslot;
-    int t = sc.cut_tile[c], jb = sc.cut_blk[c];
-    const int tend = sc.cut_tile[c + 1], bend = sc.cut_blk[c + 1];
-    while (t < tend || (t == tend && jb < bend)) {
-      const int je = t == tend ? bend : nbt[t];
-      if (jb > 0 || je < nbt[t]) {
-        if (cl.n == 0 || cl.tile[cl.n - 1] != t) {
-          if (cl.n == MAXC) return cudaErrorInvalidValue;   // at most G - 1 cuts split
-          cl.piece0[cl.n] = nslot;
-          cl.tile[cl.n++] = t;
-        }
-        ++nslot;
-      }
-      ++t;
-      jb = 0;
-    }
-  }
-  cl.piece0[cl.n] = nslot;
-  if (nslot > 2 * ncl) return cudaErrorInvalidValue;    // at most two per cluster
-  if (nslot > 0) {
-    a.ws_o = (float*)workspace;
-    a.ws_lse = a.ws_o + (size_t)2 * ncl * TM * g.Dc;
-  }
-  if (G == 0) return cudaSuccess;
 
-  if (variant == 1)
-    attend_kernel<1><<<(unsigned)(2 * G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, sc);
-  else
-    attend_kernel<0><<<(unsigned)(2 * G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, sc);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  count_launches(1);
-  if (cl.n > 0) {
-    e = launch_combine(a, cl, st);
+  // ---- batches per launch.  Every tile of a sequence reads that sequence's keys.  With
+  // all sequences in one launch, each cluster walks its own run of consecutive tiles, so
+  // the clusters spread over every sequence at once and, when the sequences' keys
+  // together crowd L2, they are read from HBM again and again.  Sequences then go in
+  // groups whose keys fit a third of L2, as long as a group's tiles still give every
+  // cluster several; groups run one after another (stream order also keeps the
+  // workspace of one group's merge apart from the next group's partials).
+  int group = g.B;
+  {
+    int dev = 0, l2 = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) == cudaSuccess && l2 > 0) {
+      const double keys_bytes = (double)n_keys * g.row * 2;     // one sequence's keys
+      if (keys_bytes * g.B > l2 / 3.0) {
+        const int by_l2 = (int)((l2 / 3.0) / keys_bytes);                  // fit a third of L2
+        const int fill = (4 * ncl + tiles_per_batch - 1) / tiles_per_batch;   // >= 4 tiles each
+        const int want = by_l2 > fill ? by_l2 : fill;
+        group = want < 1 ? 1 : (want < g.B ? want : g.B);
+      }
+    }
+  }
+
+  for (int b0 = 0; b0 < g.B; b0 += group) {
+    const int t_lo = b0 * tiles_per_batch;
+    const int t_hi = (b0 + group < g.B ? b0 + group : g.B) * tiles_per_batch;
+    const int Tg = t_hi - t_lo;
+
+    // ---- schedule: the blocks of the group's tiles end to end, one equal range per
+    // cluster (tile indices are absolute)
+    std::vector<int64_t> pre(Tg + 1, 0);
+    std::vector<int> nbt(Tg);
+    for (int t = 0; t < Tg; ++t) {
+      nbt[t] = tile_geo(g, n_q, q_first, k_first, n_keys, a.tiles_per_batch, t_lo + t, bn).blk.nblk;
+      pre[t + 1] = pre[t] + nbt[t];
+    }
+    const int64_t W = pre[Tg];
+    // Two candidate schedules, costed in key blocks: a cluster's blocks plus SEG_COST per
+    // segment it walks (the switch: Q reload, output epilogue, pipeline refill), plus
+    // COMBINE_COST when tiles are split (the merge launch).  Both costs were measured on
+    // B200 (video chunk, long window and decode shapes).
+    constexpr int64_t SEG_COST = 7, COMBINE_COST = 16;
+    // schedules below are in group-relative tiles until they are shifted for the launch
+    auto cost = [&](const Sched& c, int nc) {
+      int64_t worst = 0;
+      bool any_split = false;
+      for (int k = 0; k < nc; ++k) {
+        const int t0 = c.cut_tile[k], b0_ = c.cut_blk[k], t1 = c.cut_tile[k + 1], b1 = c.cut_blk[k + 1];
+        const int64_t blocks = (pre[t1] + b1) - (pre[t0] + b0_);
+        const int64_t segs = (int64_t)(t1 - t0) + (b1 > 0 ? 1 : 0);
+        any_split = any_split || b0_ > 0 || b1 > 0;
+        worst = blocks + SEG_COST * segs > worst ? blocks + SEG_COST * segs : worst;
+      }
+      return worst + (any_split ? COMBINE_COST : 0);
+    };
+    // cuts on tile boundaries: the first one at or past an equal share of the blocks (of
+    // the tiles when there are no blocks)
+    Sched whole{};
+    const int G_whole = Tg < ncl ? Tg : ncl;
+    {
+      int t = 0;
+      for (int c = 1; c <= G_whole; ++c) {
+        if (c == G_whole) {
+          t = Tg;
+        } else if (W > 0) {
+          const int64_t pos = W * c / G_whole;
+          while (t < Tg && pre[t] < pos) ++t;
+        } else {
+          t = (int)((int64_t)Tg * c / G_whole);
+        }
+        whole.cut_tile[c] = t;
+        whole.cut_blk[c] = 0;
+      }
+    }
+    Sched sc = whole;
+    int G = G_whole;
+    if (split && W > 0) {
+      // cut c at block W*c/G; tiles without blocks go with the range before them
+      Sched sk{};
+      const int G_split = (int)(W < ncl ? W : ncl);
+      int t = 0;
+      for (int c = 1; c <= G_split; ++c) {
+        const int64_t pos = W * c / G_split;
+        while (t < Tg && pre[t + 1] <= pos) ++t;      // tile holding block `pos`
+        sk.cut_tile[c] = t;
+        sk.cut_blk[c] = t < Tg ? (int)(pos - pre[t]) : 0;
+      }
+      if (cost(sk, G_split) < cost(whole, G_whole)) {
+        sc = sk;
+        G = G_split;
+      }
+    }
+    sc.cut_tile[0] = 0;
+    sc.cut_blk[0] = 0;
+    // partial segments: their workspace slots, and the tiles to combine
+    CombineList cl{};
+    int nslot = 0;
+    for (int c = 0; c < G; ++c) {
+      sc.slot0[c] = nslot;
+      int t = sc.cut_tile[c], jb = sc.cut_blk[c];
+      const int tend = sc.cut_tile[c + 1], bend = sc.cut_blk[c + 1];
+      while (t < tend || (t == tend && jb < bend)) {
+        const int je = t == tend ? bend : nbt[t];
+        if (jb > 0 || je < nbt[t]) {
+          if (cl.n == 0 || cl.tile[cl.n - 1] != t_lo + t) {
+            if (cl.n == MAXC) return cudaErrorInvalidValue;   // at most G - 1 cuts split
+            cl.piece0[cl.n] = nslot;
+            cl.tile[cl.n++] = t_lo + t;
+          }
+          ++nslot;
+        }
+        ++t;
+        jb = 0;
+      }
+    }
+    cl.piece0[cl.n] = nslot;
+    if (nslot > 2 * ncl) return cudaErrorInvalidValue;    // at most two per cluster
+    if (nslot > 0) {
+      a.ws_o = (float*)workspace;
+      a.ws_lse = a.ws_o + (size_t)2 * ncl * TM * g.Dc;
+    }
+    if (G == 0) continue;
+    for (int c = 0; c <= G; ++c) sc.cut_tile[c] += t_lo;
+
+    if (variant == 1)
+      attend_kernel<1><<<(unsigned)(2 * G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, sc);
+    else
+      attend_kernel<0><<<(unsigned)(2 * G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, sc);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
+    if (cl.n > 0) {
+      e = launch_combine(a, cl, st);
+      if (e != cudaSuccess) return e;
+      count_launches(1);
+    }
   }
   return cudaSuccess;
 }

@@ -66,6 +66,51 @@ def step_flops(wl) -> dict:
     }
 
 
+def step_bytes(wl) -> dict:
+    """Algorithmic HBM bytes of each call of the step: every operand read once, every
+    result written once (the attention reads the window's cached rows once)."""
+    e, T, B, H = wl.elem_bytes, wl.n_queries, wl.batch, wl.n_heads
+    return {
+        "cache_write": (B * T * wl.d_model + wl.d_model * wl.row_width + B * T * wl.row_width) * e,
+        "absorb_q": (B * T * H * (wl.d_nope + wl.d_rope) + H * wl.d_nope * wl.d_latent
+                     + B * T * H * wl.row_width) * e,
+        "attend": (B * T * H * wl.row_width + B * wl.n_keys * wl.row_width
+                   + B * T * H * wl.d_latent) * e + B * T * H * 4,
+        "up_v": (B * T * H * wl.d_latent + H * wl.d_nope * wl.d_latent + B * T * H * wl.d_nope) * e,
+    }
+
+
+def materialised_flops(wl) -> int:
+    """Flops of the non-absorbed alternative for the same attention: K and V materialised
+    once per (key, head) from the latent, then attention over d_h + d_R and d_h."""
+    mat = 2 * 2 * wl.batch * wl.n_keys * wl.n_heads * wl.d_latent * wl.d_nope
+    att = visible_pairs(wl) * wl.n_heads * (2 * (wl.d_nope + wl.d_rope) + 2 * wl.d_nope)
+    return mat + att
+
+
+def kernel_rooflines(wl, kernels_ms, peaks) -> dict:
+    """Per call of the step: achieved TFLOP/s and GB/s against the measured peaks, and the
+    bound that binds (the larger of flops/peak and bytes/bandwidth)."""
+    fl, by = step_flops(wl), step_bytes(wl)
+    tf, bw = float(peaks["bf16_tflops"]), float(peaks["hbm_gbs"])
+    out = {}
+    for k, ms in kernels_ms.items():
+        s = ms * 1e-3
+        t_tensor, t_hbm = fl[k] / (tf * 1e12), by[k] / (bw * 1e9)
+        out[k] = {"ms": ms, "flops": fl[k], "bytes": by[k],
+                  "tflops": fl[k] / s / 1e12, "frac_tensor": fl[k] / s / 1e12 / tf,
+                  "gbs": by[k] / s / 1e9, "frac_hbm": by[k] / s / 1e9 / bw,
+                  "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                  "frac_of_bound": max(t_tensor, t_hbm) / s}
+    return out
+
+
+def percentiles(xs) -> list:
+    q = sorted(xs)
+    pick = lambda f: q[min(len(q) - 1, int(round(f * (len(q) - 1))))]
+    return [pick(0.1), pick(0.5), pick(0.9)]
+
+
 def decode_bytes(wl) -> int:
     """Algorithmic bytes of one decode attention call: every cached row read once,
     q_abs read, o_lat and the LSE written."""
@@ -350,7 +395,15 @@ def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
         threads = max([i.get("num_threads", 1) for i in info] or [1])
     except Exception:  # noqa: BLE001
         threads = os.cpu_count()
+    cpu_model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            cpu_model = next((ln.split(":", 1)[1].strip() for ln in f if ln.startswith("model name")),
+                             None)
+    except OSError:
+        pass
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model, "cpu_count": os.cpu_count(),
             "sample": f"first {n_q} of {wl.n_queries} chunk queries"
                       + (f" of each of {wl.batch} sequences" if wl.batch > 1 else "")
                       + f" (all {wl.n_heads} heads, {wl.n_keys} keys): cache write, absorption, "
@@ -446,6 +499,7 @@ def run_ours(args):
     value = job_throughput(world, flops_step, args.steps, t_max) / 1e12
     peaks, peak_src = load_peaks()
     kernels_ms = {k: statistics.mean(v) for k, v in zip(Step.STAGES, parts)}
+    attend_ms_all = dict(zip(Step.STAGES, parts))["attend"]
     att_ms = kernels_ms["attend"]
     achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
@@ -472,7 +526,13 @@ def run_ours(args):
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "traffic": attend_traffic(wl), "traffic_unit": "B per launch (ncu)",
-                         "ms_per_launch": att_ms},
+                         "ms_per_launch": att_ms,
+                         "materialised_flops": materialised_flops(wl),
+                         "materialised_note": "the non-absorbed alternative's flops for the "
+                                              "same attention, for context; not what runs"},
+            "ms_percentiles": {"step_p10_p50_p90": percentiles(ms),
+                               "attend_p10_p50_p90": percentiles(attend_ms_all)},
+            "kernel_rooflines": kernel_rooflines(wl, kernels_ms, peaks),
             "e2e": {"value": job_throughput(world, flops_step, args.steps, e2e_total) / 1e12,
                     "pipelining": "upload and download streams overlap step i+1's inputs and "
                                   "step i-1's output with step i's compute; no L2 flush (a "

@@ -1,0 +1,64 @@
+"""The work accounting bench.py reports beside its timings (CPU only): algorithmic bytes per
+call, the non-absorbed alternative's flops, which roofline bound binds, and the step
+workloads the --workload option offers."""
+
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from synth import configs as C  # noqa: E402
+
+PEAKS = {"bf16_tflops": 1647.8, "hbm_gbs": 6537.3}
+
+
+def test_chunk_bytes_per_call():
+    wl = C.VIDEO_CHUNK
+    by = bench.step_bytes(wl)
+    # h [1560, 4096] + [W_DKV | W_KR] [4096, 576] read, 1560 cache rows of 576 written
+    assert by["cache_write"] == (1560 * 4096 + 4096 * 576 + 1560 * 576) * 2
+    # q_nope and q_R [1560, 32, 128 + 64] + W_UK [32, 128, 512] read, q_abs [1560, 32, 576] written
+    assert by["absorb_q"] == (1560 * 32 * 192 + 32 * 128 * 512 + 1560 * 32 * 576) * 2
+    # q_abs and the window's 6240 rows read, o_lat [1560, 32, 512] and the fp32 LSE written
+    assert by["attend"] == (1560 * 32 * 576 + 6240 * 576 + 1560 * 32 * 512) * 2 + 1560 * 32 * 4
+    assert by["up_v"] == (1560 * 32 * 512 + 32 * 128 * 512 + 1560 * 32 * 128) * 2
+
+
+def test_materialised_alternative_flops():
+    wl = C.VIDEO_CHUNK
+    # every chunk query sees all 6240 window keys; K and V materialised once per (key, head)
+    mat = 2 * 2 * 6240 * 32 * 512 * 128
+    att = 1560 * 6240 * 32 * (2 * (128 + 64) + 2 * 128)
+    assert bench.materialised_flops(wl) == mat + att
+    assert bench.materialised_flops(wl) == pytest.approx(0.2517e12, rel=1e-3)
+    # the absorbed form does more flops than the materialised one at the chunk
+    assert bench.step_flops(wl)["attend"] > 2.5 * bench.materialised_flops(wl)
+
+
+def test_binding_bound_per_call():
+    wl = C.VIDEO_CHUNK
+    ms = {"cache_write": 0.0273, "absorb_q": 0.0289, "attend": 0.6395, "up_v": 0.0226}
+    r = bench.kernel_rooflines(wl, ms, PEAKS)
+    # 7.36 GFLOP (4.5 us at peak) against 19.3 MB (3.0 us): the tensor bound binds
+    assert r["cache_write"]["bound"] == "tensor"
+    # 6.5 GFLOP against ~81 MB and ~68 MB: HBM binds
+    assert r["absorb_q"]["bound"] == "hbm"
+    assert r["up_v"]["bound"] == "hbm"
+    assert r["attend"]["bound"] == "tensor"
+    for k, v in r.items():
+        assert v["frac_of_bound"] == pytest.approx(max(v["frac_tensor"], v["frac_hbm"]))
+    # 677.8 GFLOP in 0.6395 ms
+    assert r["attend"]["tflops"] == pytest.approx(677.8 / 0.6395, rel=1e-3)
+
+
+def test_percentiles_nearest_rank():
+    assert bench.percentiles([5.0]) == [5.0, 5.0, 5.0]
+    assert bench.percentiles(list(range(1, 12))) == [2, 6, 10]
+
+
+def test_step_workloads():
+    assert bench.STEP_WORKLOADS == ("video_chunk_bf16", "long_window_bf16", "wide_key_bf16")
+    assert bench.WORKLOAD.name == "video_chunk_bf16"

@@ -204,6 +204,50 @@ mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q,
                     const void* w_uv, void* out, void* stream);
 
 /*
+ * mla_attend_materialised_workspace_size — bytes of device workspace mla_attend_materialised
+ * needs: the per-head keys and then the per-head values of every ring slot, bf16,
+ * 2 * B * S * n_h * d_nope * 2 bytes.  0 for shapes the call does not support.
+ */
+size_t mla_attend_materialised_workspace_size(const mla_shape* shape);
+
+/*
+ * mla_attend_materialised — the non-absorbed form of steps 3 and 5 together: the
+ * per-head keys and values are rebuilt from the latent ("Understanding Multi-Head
+ * Latent Attention and KV Compression", "On-the-Fly Reconstruction and Matrix
+ * Absorption"), and attention runs per head on the concatenation of the content and
+ * RoPE channels (concept page, "The RoPE problem, and the decoupled fix").  Same result
+ * as mla_absorb_q + mla_attend + mla_up_v up to rounding, with fewer flops whenever the
+ * window holds more keys than a head has dimensions to absorb (chunks, not decode).
+ *
+ * For every ring slot r of every sequence b, and head h:
+ *   K[b][r][h] = w_uk[h] . cache[b][r][0 : d_latent]     V[b][r][h] = w_uv[h] . cache[b][r][0 : d_latent]
+ * (into the workspace, rounded to bf16); then for every (b, i, h), with the keys, window
+ * and frame-block-causal mask of mla_attend:
+ *   s(g)  = softmax_scale * (q_nope[b][i][h] . K[b][g mod S][h]
+ *                            + RoPE3D(q_rope[b][i][h], position of q_first_tok + i) . cache[b][g mod S][d_latent :])
+ *   out[b][i][h] = sum_g softmax(s)(g) * V[b][g mod S][h]
+ *   lse[b][i][h] = log(sum_g exp(s(g)))   (natural log, float32; if lse != NULL)
+ *
+ *   q_nope [B, n_q, n_h, d_nope]      read
+ *   q_rope [B, n_q, n_h, d_rope]      read (un-rotated)
+ *   cache  [B, S, d_latent + d_rope]  read
+ *   w_uk, w_uv [n_h, d_nope, d_latent] read
+ *   out    [B, n_q, n_h, d_nope]      written
+ *   lse    [B, n_q, n_h] float32 or NULL written
+ *   workspace: at least mla_attend_materialised_workspace_size() bytes (required); its
+ *   contents on entry do not matter, and calls sharing one must not run concurrently.
+ * Supported: bf16 storage, d_nope = 128, d_rope = 64, d_latent a multiple of 128.
+ * Errors: those of mla_attend; MLA_ERR_UNSUPPORTED for other shapes or float32;
+ * MLA_ERR_ARG if the workspace is NULL or smaller than required.
+ */
+mla_status mla_attend_materialised(const mla_shape* shape, const void* q_nope,
+                                   const void* q_rope, int64_t n_q, int64_t q_first_tok,
+                                   const void* cache, int64_t k_first_tok, int64_t n_keys,
+                                   float softmax_scale, const void* w_uk, const void* w_uv,
+                                   void* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
  * mla_kernel_launches — number of kernels this library has launched in this process
  * (a host-side counter, incremented at every successful launch).  Diagnostic only.
  */

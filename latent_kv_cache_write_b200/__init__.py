@@ -1,6 +1,6 @@
 """Absorbed multi-head latent attention over a sliding-window latent KV ring on B200.
 
-Python face of ``libmla.so``: the four calls of the C ABI under the same names, taking
+Python face of ``libmla.so``: the calls of the C ABI under the same names, taking
 ``torch`` CUDA tensors (or raw device pointers) and enqueuing on the current CUDA
 stream unless a stream is given.  PyTorch supplies device memory and streams only;
 all arithmetic runs in the library's kernels.
@@ -15,8 +15,9 @@ from . import native
 from .native import MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
-           "mla_attend_fixed_scratch",
-           "mla_up_v", "mla_device_error", "mla_kernel_launches", "mla_device_error_info", "make_shape", "MlaShape", "MlaError"]
+           "mla_attend_fixed_scratch", "mla_attend_materialised",
+           "mla_attend_materialised_workspace_size", "mla_up_v", "mla_device_error",
+           "mla_kernel_launches", "mla_device_error_info", "make_shape", "MlaShape", "MlaError"]
 
 
 def _ptr(t) -> Optional[int]:
@@ -72,6 +73,23 @@ def mla_attend_fixed_scratch(shape: MlaShape, q_abs, n_q: int, q_first_tok: int,
     native.check("mla_attend_fixed_scratch", native.lib().mla_attend_fixed_scratch(
         ctypes.byref(shape), _ptr(q_abs), n_q, q_first_tok, _ptr(cache), k_first_tok, n_keys,
         softmax_scale, _ptr(o_lat), _ptr(lse), _stream(stream)))
+
+
+def mla_attend_materialised_workspace_size(shape: MlaShape) -> int:
+    return int(native.lib().mla_attend_materialised_workspace_size(ctypes.byref(shape)))
+
+
+def mla_attend_materialised(shape: MlaShape, q_nope, q_rope, n_q: int, q_first_tok: int,
+                            cache, k_first_tok: int, n_keys: int, softmax_scale: float, w_uk,
+                            w_uv, out, lse=None, workspace=None,
+                            workspace_bytes: Optional[int] = None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else (
+            workspace.numel() * workspace.element_size())
+    native.check("mla_attend_materialised", native.lib().mla_attend_materialised(
+        ctypes.byref(shape), _ptr(q_nope), _ptr(q_rope), n_q, q_first_tok, _ptr(cache),
+        k_first_tok, n_keys, softmax_scale, _ptr(w_uk), _ptr(w_uv), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def mla_up_v(shape: MlaShape, o_lat, n_q: int, w_uv, out, stream=None) -> None:

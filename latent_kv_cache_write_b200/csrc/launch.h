@@ -35,6 +35,17 @@ cudaError_t tc_absorb_q(const Geo& g, const void* q_nope, const void* q_rope, in
                         cudaStream_t st);
 cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_uv, void* out,
                     unsigned int* err, cudaStream_t st);
+// out[b][slot][h] = w[h] . cache[b][slot][0 : d_latent] for every ring slot (the per-head
+// keys with w = W_UK, the values with w = W_UV), bf16 [B, S, n_h, d_nope].
+cudaError_t tc_materialise(const Geo& g, const void* cache, const void* w, void* out,
+                           unsigned int* err, cudaStream_t st);
+
+// Non-absorbed attention over the materialised keys and values (tc_attend_mat.cu).
+bool tc_attend_mat_supported(const Geo& g);
+cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,
+                          int64_t q_first, const void* cache, const void* k_mat,
+                          const void* v_mat, int64_t k_first, int64_t n_keys, float scale,
+                          void* out, float* lse, unsigned int* err, cudaStream_t st);
 
 bool tc_attend_supported(const Geo& g);
 // Workspace for split-key partials on the current device (0 if it cannot be queried).

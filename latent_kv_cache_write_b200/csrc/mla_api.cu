@@ -205,6 +205,47 @@ mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, cons
   return cuda_status(simt_up_v(g, bf, o_lat, n_q, w_uv, out, (cudaStream_t)stream));
 }
 
+size_t mla_attend_materialised_workspace_size(const mla_shape* shape) {
+  Geo g;
+  if (check_shape(shape, &g) != MLA_OK) return 0;
+  if (shape->dtype != MLA_BF16 || !tc_attend_mat_supported(g) || !tc_gemm_supported(g, 0))
+    return 0;
+  return (size_t)2 * g.B * g.S * g.H * g.Dn * 2;
+}
+
+mla_status mla_attend_materialised(const mla_shape* shape, const void* q_nope,
+                                   const void* q_rope, int64_t n_q, int64_t q_first_tok,
+                                   const void* cache, int64_t k_first_tok, int64_t n_keys,
+                                   float softmax_scale, const void* w_uk, const void* w_uv,
+                                   void* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  if (n_q < 0 || !q_nope || !q_rope || !cache || !w_uk || !w_uv || !out) return MLA_ERR_ARG;
+  if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return MLA_ERR_ARG;
+  if (n_keys < 1 || n_keys > g.S || k_first_tok < 0 || q_first_tok < k_first_tok ||
+      q_first_tok + n_q > k_first_tok + n_keys)
+    return MLA_ERR_RANGE;
+  const size_t need = mla_attend_materialised_workspace_size(shape);
+  if (need == 0 || n_q > 65535) return MLA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < need) return MLA_ERR_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(cache) || !aligned16(w_uk) ||
+      !aligned16(w_uv) || !aligned16(out) || (lse && !aligned16(lse)) || !aligned16(workspace))
+    return MLA_ERR_ALIGN;
+  if (n_q == 0) return MLA_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned int* err = device_error_word();
+  uint8_t* k_mat = static_cast<uint8_t*>(workspace);
+  uint8_t* v_mat = k_mat + need / 2;
+  cudaError_t e = tc_materialise(g, cache, w_uk, k_mat, err, s);
+  if (e == cudaSuccess) e = tc_materialise(g, cache, w_uv, v_mat, err, s);
+  if (e == cudaSuccess)
+    e = tc_attend_mat(g, q_nope, q_rope, n_q, q_first_tok, cache, k_mat, v_mat, k_first_tok,
+                      n_keys, softmax_scale, out, lse, err, s);
+  return cuda_status(e);
+}
+
 void mla_device_error_info(uint32_t info[4]) {
   for (int i = 0; i < 4; ++i) info[i] = g_last_error_info[i];
 }

@@ -2,6 +2,7 @@
 //   cache write:  [h] x [W_DKV | W_KR]  -> RoPE on the W_KR columns -> bf16 -> ring slot
 //   absorb:       q_nope[:, h] x W_UK[h] -> q_lat (plus RoPE of q_R in the same CTAs)
 //   up-projection: o_lat[:, h] x W_UV[h]^T -> out
+//   materialisation: c[slot] x W[h]^T -> per-head keys or values of every ring slot
 // Persistent: one CTA per SM walks the 128 x 128 output tiles (M fastest, so CTAs that
 // run together share the weight tile in L2).  Warp 0 lane 0 streams TMA loads through a
 // 4-stage shared-memory ring, warp 1 lane 0 issues tcgen05.mma (M=128, N=128, K=16 steps)
@@ -40,7 +41,7 @@ template <int ST, bool SK> struct GLay {
   static constexpr int SMEM = OFF_OST + (SK ? 0 : 2 * OBOX_BYTES) + 1024;
 };
 
-enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2 };
+enum Mode { MODE_CACHE = 0, MODE_ABSORB = 1, MODE_UPV = 2, MODE_MAT = 3 };
 
 struct TcGemm {
   int M, N, K, Z;
@@ -145,7 +146,9 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
           uint8_t* a = smem + s * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
           mbar_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_3d(a, &tmA, &full[s], kb * GBK, p.mode == MODE_CACHE ? 0 : z, m0);
+          // the cache write's and the materialisation's A rows serve every head
+          tma_load_3d(a, &tmA, &full[s], kb * GBK,
+                      p.mode == MODE_CACHE || p.mode == MODE_MAT ? 0 : z, m0);
           if (p.b_mn) {
             tma_load_3d(b, mB, &full[s], nb, kb * GBK, z);
             tma_load_3d(b + B_BYTES / 2, mB, &full[s], nb + 64, kb * GBK, z);
@@ -582,6 +585,37 @@ cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_
   CUtensorMap O;
   {
     // out as (d_nope, heads, rows): 64-column boxes of 128 rows of one head
+    uint64_t d[3] = {(uint64_t)g.Dn, (uint64_t)g.H, rows};
+    uint64_t s[2] = {(uint64_t)g.Dn * 2, (uint64_t)g.H * g.Dn * 2};
+    uint32_t b[3] = {64, 1, (uint32_t)GBM};
+    if (!make_tmap_bf16(&O, out, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  return launch(A, B, B, O, p, g.H, st);
+}
+
+cudaError_t tc_materialise(const Geo& g, const void* cache, const void* w, void* out,
+                           unsigned int* err, cudaStream_t st) {
+  CUtensorMap A, B;
+  const uint64_t rows = (uint64_t)g.B * g.S;
+  {
+    // the latent columns of every cached row, as (d_latent, 1, slots)
+    uint64_t d[3] = {(uint64_t)g.Dc, 1, rows};
+    uint64_t s[2] = {(uint64_t)g.row * 2, (uint64_t)g.row * 2};
+    uint32_t b[3] = {64, 1, 128};
+    if (!make_tmap_bf16(&A, cache, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t d[3] = {(uint64_t)g.Dc, (uint64_t)g.Dn, (uint64_t)g.H};
+    uint64_t s[2] = {(uint64_t)g.Dc * 2, (uint64_t)g.Dc * g.Dn * 2};
+    uint32_t b[3] = {64, (uint32_t)GBN, 1};
+    if (!make_tmap_bf16(&B, w, 3, d, s, b)) return cudaErrorInvalidValue;
+  }
+  TcGemm p{};
+  p.M = (int)rows; p.N = g.Dn; p.K = g.Dc; p.mode = MODE_MAT; p.b_mn = 0;
+  p.n_split = 1 << 30; p.out = (bf16*)out; p.rows_per_batch = g.S; p.geo = g; p.err = err;
+  CUtensorMap O;
+  {
+    // out as (d_nope, heads, slots): 64-column boxes of 128 slots of one head
     uint64_t d[3] = {(uint64_t)g.Dn, (uint64_t)g.H, rows};
     uint64_t s[2] = {(uint64_t)g.Dn * 2, (uint64_t)g.H * g.Dn * 2};
     uint32_t b[3] = {64, 1, (uint32_t)GBM};

@@ -134,3 +134,32 @@ def test_absorb_and_up_v_validation(L):
     assert uv(w=ODD) == native.MLA_ERR_ALIGN
     assert uv(n=-2) == native.MLA_ERR_ARG
     assert uv(n=0) == native.MLA_OK
+
+
+def _mat(L, s, qn=FAKE, qr=FAKE, n_q=1560, q_first=3 * 1560, cache=FAKE, k_first=0,
+         n_keys=6240, scale=0.07, wuk=FAKE, wuv=FAKE, out=FAKE, lse=None, ws=FAKE,
+         ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = L.mla_attend_materialised_workspace_size(ctypes.byref(s))
+    return L.mla_attend_materialised(ctypes.byref(s), qn, qr, n_q, q_first, cache, k_first,
+                                     n_keys, scale, wuk, wuv, out, lse, ws, ws_bytes, None)
+
+
+def test_materialised_validation(L):
+    s = _shape()
+    # per-head keys and values of every ring slot, bf16
+    assert L.mla_attend_materialised_workspace_size(ctypes.byref(s)) == 2 * 6240 * 32 * 128 * 2
+    wide = native.make_shape(C.WIDE_KEY)
+    assert L.mla_attend_materialised_workspace_size(ctypes.byref(wide)) == 0
+    assert _mat(L, wide, n_q=1560, q_first=9 * 1560, n_keys=15600, ws_bytes=1 << 30) == \
+        native.MLA_ERR_UNSUPPORTED
+    assert _mat(L, _shape(dtype=native.MLA_F32), ws_bytes=1 << 30) == native.MLA_ERR_UNSUPPORTED
+    assert _mat(L, s, ws=None) == native.MLA_ERR_ARG
+    assert _mat(L, s, ws_bytes=1024) == native.MLA_ERR_ARG
+    assert _mat(L, s, qr=None) == native.MLA_ERR_ARG
+    assert _mat(L, s, wuv=None) == native.MLA_ERR_ARG
+    assert _mat(L, s, n_keys=6241) == native.MLA_ERR_RANGE
+    assert _mat(L, s, q_first=3 * 1560 + 1) == native.MLA_ERR_RANGE
+    assert _mat(L, s, out=ODD) == native.MLA_ERR_ALIGN
+    assert _mat(L, s, ws=ODD) == native.MLA_ERR_ALIGN
+    assert _mat(L, s, n_q=0, q_first=0) == native.MLA_OK          # empty: nothing to do

@@ -328,6 +328,38 @@ def time_steps(torch, fn, steps, flush, n_marks=0):
     return st, parts
 
 
+def materialised_leg(torch, mla, step, steps, warmup, flush, absorbed_ms):
+    """The non-absorbed form of the same chunk: mla_attend_materialised (the per-head keys
+    and values rebuilt from the latent, then attention in head space, output up-projected)
+    on the step's queries and cache; it replaces the absorption, the absorbed attention and
+    the up-projection of the step."""
+    wl = step.wl
+    if mla.mla_attend_materialised_workspace_size(step.shape) == 0:
+        return None
+    T = wl.n_queries
+    nws = mla.mla_attend_materialised_workspace_size(step.shape)
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(step.out)
+    lse = torch.empty_like(step.lse)
+
+    def call(_a=None):
+        mla.mla_attend_materialised(step.shape, step.dev_in["q_nope"], step.dev_in["q_rope"], T,
+                                    wl.q_first_tok, step.cache, wl.k_first_tok, wl.n_keys,
+                                    wl.softmax_scale, step.w["w_uk"], step.w["w_uv"], out, lse,
+                                    ws, nws)
+
+    for _ in range(warmup):
+        call()
+    ms, _ = time_steps(torch, call, steps, flush)
+    t = statistics.mean(ms)
+    fl = materialised_flops(wl)
+    return {"call": "mla_attend_materialised", "ms": t, "flops": fl,
+            "tflops": fl / (t * 1e-3) / 1e12,
+            "replaces_ms": absorbed_ms, "speedup_vs_absorbed": absorbed_ms / t,
+            "note": "per-head K and V of every ring slot rebuilt, then attention in head "
+                    "space; replaces absorb_q + attend + up_v of the step"}
+
+
 def decode_leg(torch, mla, steps, warmup, flush):
     wl = C.DECODE
     shape = mla.make_shape(wl)
@@ -504,6 +536,11 @@ def run_ours(args):
     achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     dec = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush) if rank == 0 else None
+    mat = materialised_leg(torch, mla, step, max(3, args.steps), args.warmup, flush,
+                           kernels_ms["absorb_q"] + kernels_ms["attend"] + kernels_ms["up_v"]) \
+        if rank == 0 else None
+    if mat:
+        mat["frac"] = mat["tflops"] / float(peaks["bf16_tflops"])
     if dec:
         dec["peak_gbs"] = float(peaks["hbm_gbs"])
         dec["frac"] = dec["value"] / dec["peak_gbs"]
@@ -543,6 +580,7 @@ def run_ours(args):
                     "ms_per_step": e2e_total / args.steps},
             "gpu_launches": int(launches),
             "decode": dec,
+            "materialised": mat,
             "clocks": clocks.summary(),
             "kernels_ms": kernels_ms,
         }

@@ -360,8 +360,7 @@ def materialised_leg(torch, mla, step, steps, warmup, flush, absorbed_ms):
                     "space; replaces absorb_q + attend + up_v of the step"}
 
 
-def decode_leg(torch, mla, steps, warmup, flush):
-    wl = C.DECODE
+def decode_leg(torch, mla, steps, warmup, flush, wl=C.DECODE):
     shape = mla.make_shape(wl)
     dev = "cuda"
     cache = torch.from_numpy(G.direct_cache(wl, 0).storage.view(np.int16)).to(dev).view(
@@ -536,6 +535,12 @@ def run_ours(args):
     achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     dec = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush) if rank == 0 else None
+    if dec:
+        # small-batch decode: one sequence, its keys split over every cluster
+        one = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush,
+                         C.DECODE.scaled(name="decode_one_sequence", batch=1))
+        dec["one_sequence"] = {"ms": one["ms"], "value": one["value"], "unit": "GB/s",
+                               "bytes": one["bytes"]}
     mat = materialised_leg(torch, mla, step, max(3, args.steps), args.warmup, flush,
                            kernels_ms["absorb_q"] + kernels_ms["attend"] + kernels_ms["up_v"]) \
         if rank == 0 else None

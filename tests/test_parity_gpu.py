@@ -230,9 +230,11 @@ SPLIT_CHUNK = C.small_variant(C.VIDEO_CHUNK).scaled(
     first_chunk_frame=38, ring_slots=39 * 66)
 SPLIT_DECODE = C.small_variant(C.DECODE).scaled(
     name="decode_split", batch=8, ring_slots=4096, window_frames=4095, first_chunk_frame=4095)
+# small-batch decode: one sequence's 8192 keys are one tile, spread over every cluster
+DECODE_ONE = C.DECODE.scaled(name="decode_one_sequence", batch=1)
 
 
-@pytest.mark.parametrize("wl", [SPLIT_CHUNK, SPLIT_DECODE], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [SPLIT_CHUNK, SPLIT_DECODE, DECODE_ONE], ids=lambda w: w.name)
 @pytest.mark.parametrize("use_ws", [True, False], ids=["workspace", "no_workspace"])
 def test_schedule_split_and_whole(cuda_ok, wl, use_ws):
     """With a workspace these shapes cut tiles between clusters (the merge kernel runs:

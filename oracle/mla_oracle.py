@@ -18,6 +18,9 @@ Sources, cited by page title and section:
   Absorption" (per-head K and V are reconstructed from the latent with
   up-projections) and "Decoupling Rotary Position Embeddings (RoPE)" (the cache
   stores the latent alongside the RoPE key; the two key parts are concatenated).
+* [Irminsul]      the Irminsul abstract on the "Multi-Head Latent Attention" topic page:
+  the cached row is a position-free latent plus a RoPE key that a delta-rotation
+  re-indexes in closed form when the same tokens move to shifted positions.
 * [VideoMLA]      "VideoMLA: Compressing Video Diffusion Memory by 92.7% with
   Low-Rank Latent Attention", sections "The Gap" (sliding-window KV cache,
   next-frame prediction) and "Core Mechanism" (a shared content latent and a
@@ -146,6 +149,24 @@ def cache_write(cache: np.ndarray, h: np.ndarray, w_dkv: np.ndarray, w_kr: np.nd
             out[b, s] = rows[b, i]
             slots[b, i] = s
     return out, slots
+
+
+def shift_frames(cache: np.ndarray, first_tok: int, n_tok: int, delta_frames: int,
+                 wl) -> np.ndarray:
+    """Re-index cached RoPE keys to positions delta_frames frames later ([Irminsul]
+    delta-rotation; [VideoMLA] "Core Mechanism" for the 3-D positions).
+
+    A whole-frame shift moves t by delta_frames and leaves y and x alone, so the RoPE
+    key of each token g in [first_tok, first_tok + n_tok) (slot g mod S) is turned by
+    the angles of position (delta_frames, 0, 0); the latent is position-free and stays.
+    Returns a new cache."""
+    out = np.array(cache, dtype=np.float64, copy=True)
+    d_c = wl.d_latent
+    ang = rope_angles(delta_frames, 0, 0, wl.rope_pairs, wl.rope_theta)
+    for g in range(first_tok, first_tok + n_tok):
+        slot = ring_slot(g, wl.ring_slots)
+        out[:, slot, d_c:] = rotate_pairs(out[:, slot, d_c:], ang)
+    return out
 
 
 # ----------------------------------------------------------------------------------

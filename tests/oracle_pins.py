@@ -384,6 +384,30 @@ def pin_ring_slots():
         assert np.array_equal(cache[:, s], O.cache_rows(h, w["w_dkv"], w["w_kr"], last, wl)[:, 0])
 
 
+def pin_frame_shift():
+    """Re-indexing cached RoPE keys by whole frames equals writing the same hidden states
+    at the shifted positions (rotations compose: R(p + d) = R(d) R(p), and a shift by
+    whole frames changes t only), leaves the latent untouched, and shifting back
+    restores the rows."""
+    wl = SMALL
+    w = {k: v.values for k, v in G.weights(wl, 0).items()}
+    F = wl.tokens_per_frame
+    h = G.hidden_frame(wl, 0, 1).values                   # one frame of hidden states
+    first = 1 * F
+    for delta in (2, -1, 5):
+        cache = np.zeros((wl.batch, wl.ring_slots, wl.row_width))
+        cache, _ = O.cache_write(cache, h, w["w_dkv"], w["w_kr"], first, wl)
+        shifted = O.shift_frames(cache, first, F, delta, wl)
+        direct = O.cache_rows(h, w["w_dkv"], w["w_kr"], first + delta * F, wl)
+        slots = [g % wl.ring_slots for g in range(first, first + F)]
+        assert rel(shifted[:, slots], direct) < 1e-12, delta
+        assert np.array_equal(shifted[:, slots, :wl.d_latent], cache[:, slots, :wl.d_latent])
+        back = O.shift_frames(shifted, first, F, -delta, wl)
+        assert rel(back, cache) < 1e-12
+        others = [s for s in range(wl.ring_slots) if s not in slots]
+        assert np.array_equal(shifted[:, others], cache[:, others])
+
+
 # ---------------------------------------------------------------- C1, C2 closed forms
 
 
@@ -431,4 +455,4 @@ def pin_flop_counts():
 ALL_PINS = [pin_absorption_identity, pin_rope_relative, pin_rope_textbook_1d,
             pin_rope_axes, pin_rope_in_cache_and_query, pin_brute_force,
             pin_library_sdpa, pin_degenerate_cases, pin_mask_isolation,
-            pin_ring_slots, pin_cache_bytes, pin_flop_counts]
+            pin_ring_slots, pin_frame_shift, pin_cache_bytes, pin_flop_counts]

@@ -10,7 +10,7 @@ from tests import oracle_pins as P
 _orig = {n: getattr(O, n) for n in (
     "rotate_pairs", "rope_angles", "token_position", "visible_keys", "attend_latent",
     "attend_materialised", "absorb_q", "ring_slot", "up_v", "cache_rows", "_softmax_lse",
-    "mla_bytes_per_token", "rope3d")}
+    "mla_bytes_per_token", "rope3d", "shift_frames")}
 
 
 def _rot_sign(v, angles):
@@ -86,6 +86,20 @@ def _bytes_no_rope(d_latent, d_rope, elem_bytes):
     return d_latent * elem_bytes
 
 
+def _shift_row_axis(cache, first_tok, n_tok, delta_frames, wl):
+    # turns the y pairs instead of the t pairs
+    out = np.array(cache, dtype=np.float64, copy=True)
+    ang = O.rope_angles(0, delta_frames, 0, wl.rope_pairs, wl.rope_theta)
+    for g in range(first_tok, first_tok + n_tok):
+        s = g % wl.ring_slots
+        out[:, s, wl.d_latent:] = O.rotate_pairs(out[:, s, wl.d_latent:], ang)
+    return out
+
+
+def _shift_backwards(cache, first_tok, n_tok, delta_frames, wl):
+    return _orig["shift_frames"](cache, first_tok, n_tok, -delta_frames, wl)
+
+
 MUTATIONS = {
     "rotation_sign": ("rotate_pairs", _rot_sign),
     "rope_frequency_exponent": ("rope_angles", _angles_exp),
@@ -101,6 +115,8 @@ MUTATIONS = {
     "k_rope_single_position": ("cache_rows", _rows_one_position),
     "lse_missing_max": ("_softmax_lse", _lse_no_max),
     "cache_bytes_drop_rope": ("mla_bytes_per_token", _bytes_no_rope),
+    "shift_turns_row_axis": ("shift_frames", _shift_row_axis),
+    "shift_backwards": ("shift_frames", _shift_backwards),
 }
 
 

@@ -360,6 +360,27 @@ def materialised_leg(torch, mla, step, steps, warmup, flush, absorbed_ms):
                     "space; replaces absorb_q + attend + up_v of the step"}
 
 
+def shift_leg(torch, mla, step, steps, warmup, flush):
+    """Whole-frame re-indexing of the window's cached RoPE keys (mla_cache_shift_frames),
+    forward and back by one frame per call pair so the ring stays valid."""
+    wl = step.wl
+    n = wl.n_keys
+
+    def call(_a=None):
+        mla.mla_cache_shift_frames(step.shape, step.cache, wl.k_first_tok, n, 1)
+        mla.mla_cache_shift_frames(step.shape, step.cache, wl.k_first_tok, n, -1)
+
+    for _ in range(warmup):
+        call()
+    ms, _ = time_steps(torch, call, steps, flush)
+    t = statistics.mean(ms) / 2                       # per call
+    moved = 2 * wl.batch * n * 2 * wl.rope_pairs[0] * wl.elem_bytes     # read + write
+    return {"call": "mla_cache_shift_frames", "rows": wl.batch * n, "ms": t, "bytes": moved,
+            "value": moved / (t * 1e-3) / 1e9, "unit": "GB/s",
+            "note": "the window's t-axis RoPE pairs turned in place; a few hundred KB, so "
+                    "launch-bound"}
+
+
 def decode_leg(torch, mla, steps, warmup, flush, wl=C.DECODE):
     shape = mla.make_shape(wl)
     dev = "cuda"
@@ -546,6 +567,8 @@ def run_ours(args):
         if rank == 0 else None
     if mat:
         mat["frac"] = mat["tflops"] / float(peaks["bf16_tflops"])
+    shift = shift_leg(torch, mla, step, max(3, args.steps), args.warmup, flush) \
+        if rank == 0 else None
     if dec:
         dec["peak_gbs"] = float(peaks["hbm_gbs"])
         dec["frac"] = dec["value"] / dec["peak_gbs"]
@@ -586,6 +609,7 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "decode": dec,
             "materialised": mat,
+            "k_rope_shift": shift,
             "clocks": clocks.summary(),
             "kernels_ms": kernels_ms,
         }

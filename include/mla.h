@@ -204,6 +204,29 @@ mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q,
                     const void* w_uv, void* out, void* stream);
 
 /*
+ * mla_cache_shift_frames — whole-frame re-indexing of cached RoPE keys (the
+ * delta-rotation for reused tokens at shifted positions, Irminsul abstract on the
+ * "Multi-Head Latent Attention" topic page; positions as in VideoMLA "Core Mechanism").
+ *
+ * For b < B and the ring slots g mod S of g = first_tok .. first_tok + n_tok - 1, turn the
+ * cached RoPE key as if its token had been written delta_frames frames later (or earlier,
+ * for a negative delta_frames):
+ *   cache[b][g mod S][d_latent : +d_rope] = RoPE3D-rotation by position (delta_frames, 0, 0)
+ * A frame shift changes t only: the t-axis pairs turn by delta_frames * theta^(-j/n_t); the
+ * y and x pairs and the latent are left as they are.  A row written for token g therefore
+ * equals, up to rounding, what mla_cache_write stores for token g + delta_frames * F.  In
+ * place: the rows stay in their slots, and the caller keeps track of the positions they
+ * now stand for (shifts compose; a shift by a whole ring, delta_frames * F a multiple of S,
+ * keeps the slot convention g mod S).
+ *
+ *   cache [B, S, d_latent + d_rope]   read and written at n_tok slots
+ * Errors: MLA_ERR_RANGE if n_tok > S or first_tok < 0; MLA_ERR_ARG for a NULL cache or
+ * n_tok < 0.
+ */
+mla_status mla_cache_shift_frames(const mla_shape* shape, void* cache, int64_t first_tok,
+                                  int64_t n_tok, int64_t delta_frames, void* stream);
+
+/*
  * mla_attend_materialised_workspace_size — bytes of device workspace mla_attend_materialised
  * needs: the per-head keys and then the per-head values of every ring slot, bf16,
  * 2 * B * S * n_h * d_nope * 2 bytes.  0 for shapes the call does not support.

@@ -15,7 +15,7 @@ from . import native
 from .native import MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
-           "mla_attend_fixed_scratch", "mla_attend_materialised",
+           "mla_attend_fixed_scratch", "mla_attend_materialised", "mla_cache_shift_frames",
            "mla_attend_materialised_workspace_size", "mla_up_v", "mla_device_error",
            "mla_kernel_launches", "mla_device_error_info", "make_shape", "MlaShape", "MlaError"]
 
@@ -73,6 +73,12 @@ def mla_attend_fixed_scratch(shape: MlaShape, q_abs, n_q: int, q_first_tok: int,
     native.check("mla_attend_fixed_scratch", native.lib().mla_attend_fixed_scratch(
         ctypes.byref(shape), _ptr(q_abs), n_q, q_first_tok, _ptr(cache), k_first_tok, n_keys,
         softmax_scale, _ptr(o_lat), _ptr(lse), _stream(stream)))
+
+
+def mla_cache_shift_frames(shape: MlaShape, cache, first_tok: int, n_tok: int,
+                           delta_frames: int, stream=None) -> None:
+    native.check("mla_cache_shift_frames", native.lib().mla_cache_shift_frames(
+        ctypes.byref(shape), _ptr(cache), first_tok, n_tok, delta_frames, _stream(stream)))
 
 
 def mla_attend_materialised_workspace_size(shape: MlaShape) -> int:

@@ -40,6 +40,11 @@ cudaError_t tc_up_v(const Geo& g, const void* o_lat, int64_t n_q, const void* w_
 cudaError_t tc_materialise(const Geo& g, const void* cache, const void* w, void* out,
                            unsigned int* err, cudaStream_t st);
 
+// Turn the cached RoPE keys of tokens first_tok .. + n_tok by a (delta_frames, 0, 0)
+// position (rope_shift.cu).
+cudaError_t shift_frames(const Geo& g, bool bf, void* cache, int64_t first_tok, int64_t n_tok,
+                         int64_t delta_frames, cudaStream_t st);
+
 // Non-absorbed attention over the materialised keys and values (tc_attend_mat.cu).
 bool tc_attend_mat_supported(const Geo& g);
 cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,

@@ -205,6 +205,19 @@ mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, cons
   return cuda_status(simt_up_v(g, bf, o_lat, n_q, w_uv, out, (cudaStream_t)stream));
 }
 
+mla_status mla_cache_shift_frames(const mla_shape* shape, void* cache, int64_t first_tok,
+                                  int64_t n_tok, int64_t delta_frames, void* stream) {
+  Geo g;
+  mla_status st = check_shape(shape, &g);
+  if (st != MLA_OK) return st;
+  if (!cache || n_tok < 0) return MLA_ERR_ARG;
+  if (first_tok < 0 || n_tok > g.S) return MLA_ERR_RANGE;
+  if (!aligned16(cache)) return MLA_ERR_ALIGN;
+  if (n_tok == 0) return MLA_OK;
+  return cuda_status(shift_frames(g, shape->dtype == MLA_BF16, cache, first_tok, n_tok,
+                                  delta_frames, (cudaStream_t)stream));
+}
+
 size_t mla_attend_materialised_workspace_size(const mla_shape* shape) {
   Geo g;
   if (check_shape(shape, &g) != MLA_OK) return 0;

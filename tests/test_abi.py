@@ -163,3 +163,16 @@ def test_materialised_validation(L):
     assert _mat(L, s, out=ODD) == native.MLA_ERR_ALIGN
     assert _mat(L, s, ws=ODD) == native.MLA_ERR_ALIGN
     assert _mat(L, s, n_q=0, q_first=0) == native.MLA_OK          # empty: nothing to do
+
+
+def test_shift_frames_validation(L):
+    s = _shape()
+    sh = lambda **k: L.mla_cache_shift_frames(ctypes.byref(s), k.get("cache", FAKE),
+                                              k.get("first", 1560), k.get("n", 1560),
+                                              k.get("d", 2), None)
+    assert sh(cache=None) == native.MLA_ERR_ARG
+    assert sh(n=-1) == native.MLA_ERR_ARG
+    assert sh(n=6241) == native.MLA_ERR_RANGE                 # more tokens than slots
+    assert sh(first=-1) == native.MLA_ERR_RANGE
+    assert sh(cache=ODD) == native.MLA_ERR_ALIGN
+    assert sh(n=0) == native.MLA_OK                             # empty: nothing to do

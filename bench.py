@@ -468,12 +468,12 @@ def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
 # profiles/combine_kernel_video_chunk.md (the split-key merge).  Counters describe the kernel
 # sources they were taken on: the value is reported only while those sources are unchanged.
 ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
-                  "bytes": (73_877_504 + 34_028_032) + (37_907_968 + 16_896),
+                  "bytes": (73_877_504 + 34_028_032) + (37_908_480 + 28_416),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
                           "209c6e02806d9eb047d09790a18b63f7e033957a9b3a4eff799a83b980ddf56d",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
-                          "67947231c23dc78cb22b69f230758b971516c21f6b7bbc699d9acefd11dc1ca6"}}
+                          "22fa5edab23e55d50e763e652e2786bd7929fc0104daa8add48cc20ba47c7546"}}
 
 
 def attend_traffic(wl=WORKLOAD):

@@ -165,6 +165,22 @@ def test_full_sampled_rows(full_run):
     P.tol_check(P.download(r.out[b_idx, i_idx]), ref_o, wl.dtype, "out sampled")
 
 
+def test_full_attend_repeatable_and_launches(full_run):
+    """A second call gives bit-identical o_lat and lse (fixed schedule and merge order).
+    The wide-key workload's four sequences each hold 32 MB of keys, more than a third of
+    L2 together, so the call runs one attention launch per sequence (plus any merges);
+    the single-sequence chunk shapes and decode run one."""
+    r = full_run
+    wl = r.wl
+    o, lse, launches = _attend(r, wl, True)
+    assert np.array_equal(o, P.download(r.o_lat))
+    assert np.array_equal(lse, r.lse.cpu().numpy())
+    if wl is C.WIDE_KEY:
+        assert 4 <= launches <= 8, launches
+    else:
+        assert launches in (1, 2), launches
+
+
 # ------------------------------------------------------------------ edge cases
 
 

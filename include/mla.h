@@ -119,7 +119,7 @@ mla_status mla_absorb_q(const mla_shape* shape, const void* q_nope, const void* 
 
 /*
  * mla_attend_workspace_size — bytes of device workspace that lets mla_attend split the
- * key range of a tile across SMs (split-key partial outputs, float32, and their
+ * key range of a tile across SMs (split-key partial outputs, bfloat16, and their float32
  * log-sum-exps, two slots per resident cluster of the current device).  May be 0 (the
  * float32 path, and shapes without the tensor-core kernel, never need one).
  */
@@ -167,10 +167,11 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
  * For callers that cannot hand mla_attend a device workspace: a plain C host that
  * holds only the tensors it was given and no device allocator of its own, or a serving
  * loop that must not allocate between steps (cudaMalloc and cudaFree synchronise the
- * device).  Instead of the workspace, the split-key partials (float32 partial outputs
- * and log-sum-exps) go to one static device array of MLA_FIXED_SCRATCH_BYTES inside the
- * library, 40 MiB per device (two partial slots of 128 x (d_latent + 2) floats for each
- * resident pair of SMs: 37 MiB on a 148-SM B200).  The call allocates nothing.
+ * device).  Instead of the workspace, the split-key partials (bfloat16 partial outputs
+ * and float32 log-sum-exps) go to one static device array of MLA_FIXED_SCRATCH_BYTES
+ * inside the library, 40 MiB per device (two partial slots of 128 x d_latent bfloat16 and
+ * 256 floats for each resident pair of SMs: 19 MiB on a 148-SM B200, 33 MiB for the
+ * largest schedule of 128 clusters).  The call allocates nothing.
  *
  * Arguments, results and errors are those of mla_attend (without workspace and
  * workspace_bytes); the results equal mla_attend's with a full workspace.  In addition:

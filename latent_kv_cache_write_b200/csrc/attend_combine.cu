@@ -1,6 +1,6 @@
 // Merge of the split-key partials of the tensor-core attention: a tile whose key blocks
-// were cut between clusters left one normalised fp32 partial output and one log-sum-exp
-// per CTA half for each piece in the workspace.
+// were cut between clusters left one normalised bf16 partial output and one fp32
+// log-sum-exp per CTA half for each piece in the workspace.
 #include "attend_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -51,15 +51,18 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int q = 0; q < 16; ++q) acc[q] = 0.f;
   float wsum = 0.f;
-  auto add = [&](float lp, const float4 (&v)[4]) {
+  // a piece's 16 dims of this lane: two 16-byte vectors of bf16
+  auto add = [&](float lp, const uint4 (&v)[2]) {
     const float w = lp > -INFINITY ? expf(lp - mx) : 0.f;
     wsum += w;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      acc[4 * q] += w * v[q].x;
-      acc[4 * q + 1] += w * v[q].y;
-      acc[4 * q + 2] += w * v[q].z;
-      acc[4 * q + 3] += w * v[q].w;
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t u[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[8 * q + 2 * e] += w * __uint_as_float(u[e] << 16);
+        acc[8 * q + 2 * e + 1] += w * __uint_as_float(u[e] & 0xffff0000u);
+      }
     }
   };
   if (row_ok && mx > -INFINITY) {
@@ -67,25 +70,25 @@ __global__ void __launch_bounds__(256)
     if constexpr (CSPLIT > 1) {
       for (; p + 3 * CSPLIT < p1; p += 4 * CSPLIT) {
         float lp[4];
-        float4 v[4][4];
+        uint4 v[4][2];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int pu = p + u * CSPLIT;
           lp[u] = lse_h[(int64_t)pu * 2 * TM];
-          const float4* o =
-              reinterpret_cast<const float4*>(a.ws_o + ((int64_t)pu * TM + r) * a.g.Dc + d);
+          const uint4* o =
+              reinterpret_cast<const uint4*>(a.ws_o + ((int64_t)pu * TM + r) * a.g.Dc + d);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) v[u][q] = o[q];
+          for (int q = 0; q < 2; ++q) v[u][q] = o[q];
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) add(lp[u], v[u]);
       }
     }
     for (; p < p1; p += CSPLIT) {
-      float4 v[4];
-      const float4* o = reinterpret_cast<const float4*>(a.ws_o + ((int64_t)p * TM + r) * a.g.Dc + d);
+      uint4 v[2];
+      const uint4* o = reinterpret_cast<const uint4*>(a.ws_o + ((int64_t)p * TM + r) * a.g.Dc + d);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = o[q];
+      for (int q = 0; q < 2; ++q) v[q] = o[q];
       add(lse_h[(int64_t)p * 2 * TM], v);
     }
   }

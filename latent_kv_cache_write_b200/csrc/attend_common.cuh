@@ -18,7 +18,7 @@ struct AttnArgs {
   const bf16* q_abs;
   bf16* o_lat;
   float* lse;
-  float* ws_o;              // partial outputs [slot][TM][Dc], fp32, normalised by their l
+  bf16* ws_o;               // partial outputs [slot][TM][Dc], bf16, normalised by their l
   float* ws_lse;            // their natural log-sum-exps, one per CTA half [slot][2][TM]
   int tiles_per_batch;
   int bn;                   // keys per block of the launch

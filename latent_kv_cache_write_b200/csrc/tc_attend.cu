@@ -665,14 +665,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         if (!row_valid) continue;
         if (part) {
-          float4* dst = reinterpret_cast<float4*>(a.ws_o + ((int64_t)sw.slot * TM + t) * G.Dc +
-                                                  rank * HALF + c);
+          // the normalised partial, rounded to bf16 like a final output (the merge adds the
+          // pieces of a row in fp32)
+          uint4* dst = reinterpret_cast<uint4*>(a.ws_o + ((int64_t)sw.slot * TM + t) * G.Dc +
+                                                rank * HALF + c);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv,
-                                 __uint_as_float(v[4 * q + 1]) * inv,
-                                 __uint_as_float(v[4 * q + 2]) * inv,
-                                 __uint_as_float(v[4 * q + 3]) * inv);
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(
+                pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv),
+                pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv),
+                pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv),
+                pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv));
         } else {
           bf16* dst = a.o_lat + grow * G.Dc + rank * HALF + c;
 #pragma unroll
@@ -751,7 +754,8 @@ int cluster_slots() {
   return n;
 }
 
-size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc + 2) * sizeof(float); }
+// one partial slot: 128 rows of d_latent bf16 outputs and two fp32 log-sum-exps
+size_t slot_bytes(const Geo& g) { return (size_t)TM * ((size_t)g.Dc * 2 + 2 * sizeof(float)); }
 
 }  // namespace
 
@@ -918,8 +922,8 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     cl.piece0[cl.n] = nslot;
     if (nslot > 2 * ncl) return cudaErrorInvalidValue;    // at most two per cluster
     if (nslot > 0) {
-      a.ws_o = (float*)workspace;
-      a.ws_lse = a.ws_o + (size_t)2 * ncl * TM * g.Dc;
+      a.ws_o = (bf16*)workspace;
+      a.ws_lse = reinterpret_cast<float*>(a.ws_o + (size_t)2 * ncl * TM * g.Dc);
     }
     if (G == 0) continue;
     for (int c = 0; c <= G; ++c) sc.cut_tile[c] += t_lo;

@@ -468,12 +468,12 @@ def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
 # profiles/combine_kernel_video_chunk.md (the split-key merge).  Counters describe the kernel
 # sources they were taken on: the value is reported only while those sources are unchanged.
 ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
-                  "bytes": (73_877_504 + 34_028_032) + (37_908_480 + 28_416),
+                  "bytes": (72_767_232 + 18_537_728) + (19_032_576 + 0),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
-                          "209c6e02806d9eb047d09790a18b63f7e033957a9b3a4eff799a83b980ddf56d",
+                          "fac888e6957e39e953f1966007b9ff7fc03aa2ef3de6fd647d59beafc935e87a",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
-                          "22fa5edab23e55d50e763e652e2786bd7929fc0104daa8add48cc20ba47c7546"}}
+                          "8470448cc9cefd6bf7baa6b11f034bb548d5ccce3f5dfaf611570447dd93f53a"}}
 
 
 def attend_traffic(wl=WORKLOAD):

@@ -289,6 +289,16 @@ const char* mla_status_string(mla_status status);
 mla_status mla_device_error(void* stream);
 
 /*
+ * mla_check_wait_timeout — diagnostic of the failure path: enqueues one kernel whose single
+ * thread waits, with the bounded wait every tensor-core kernel of the library uses, on a
+ * barrier that nothing completes.  The wait gives up after its limit (about 2 s), records
+ * site 0x7FF in the device error word and the kernel returns; mla_device_error on the same
+ * stream then returns MLA_ERR_TIMEOUT, and the device stays usable.  Returns the launch
+ * status (MLA_OK, or MLA_ERR_CUDA).
+ */
+mla_status mla_check_wait_timeout(void* stream);
+
+/*
  * mla_device_error_info — details of the last device-side error that mla_device_error
  * reported: info[0] status bits, info[1] id of the first wait site that gave up,
  * info[2] its CTA index, info[3] a (thread << 16 | block) tag.  Zeros if none yet.

@@ -17,7 +17,8 @@ from .native import MlaError, MlaShape, make_shape  # noqa: F401
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
            "mla_attend_fixed_scratch", "mla_attend_materialised", "mla_cache_shift_frames",
            "mla_attend_materialised_workspace_size", "mla_up_v", "mla_device_error",
-           "mla_kernel_launches", "mla_device_error_info", "make_shape", "MlaShape", "MlaError"]
+           "mla_kernel_launches", "mla_device_error_info", "mla_check_wait_timeout", "make_shape",
+           "MlaShape", "MlaError"]
 
 
 def _ptr(t) -> Optional[int]:
@@ -114,6 +115,12 @@ def mla_device_error_info() -> list:
     buf = (ctypes.c_uint32 * 4)()
     native.lib().mla_device_error_info(buf)
     return list(buf)
+
+
+def mla_check_wait_timeout(stream=None) -> None:
+    """Enqueue the diagnostic whose bounded wait must expire; mla_device_error on the same
+    stream then reports MLA_ERR_TIMEOUT."""
+    native.check("mla_check_wait_timeout", native.lib().mla_check_wait_timeout(_stream(stream)))
 
 
 def mla_device_error(stream=None) -> int:

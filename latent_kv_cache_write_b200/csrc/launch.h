@@ -65,6 +65,10 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
 // Address of the static split-key scratch (MLA_FIXED_SCRATCH_BYTES) on the current device.
 cudaError_t fixed_scratch(void** ptr);
 
+// Launch one thread whose bounded wait on a barrier nothing completes must expire
+// (wait_check.cu).
+cudaError_t wait_check(unsigned int* err, cudaStream_t st);
+
 // Device address of the library's error word on the current device (nullptr on failure).
 unsigned int* device_error_word();
 

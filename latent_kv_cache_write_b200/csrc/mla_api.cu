@@ -259,6 +259,12 @@ mla_status mla_attend_materialised(const mla_shape* shape, const void* q_nope,
   return cuda_status(e);
 }
 
+mla_status mla_check_wait_timeout(void* stream) {
+  unsigned int* err = device_error_word();
+  if (!err) return MLA_ERR_CUDA;
+  return cuda_status(wait_check(err, (cudaStream_t)stream));
+}
+
 void mla_device_error_info(uint32_t info[4]) {
   for (int i = 0; i < 4; ++i) info[i] = g_last_error_info[i];
 }

@@ -46,6 +46,7 @@ SIGNATURES = {
                                        _vp, _vp, _vp, _sz, _vp]),
     "mla_status_string": (ctypes.c_char_p, [_i32]),
     "mla_device_error": (_i32, [_vp]),
+    "mla_check_wait_timeout": (_i32, [_vp]),
     "mla_kernel_launches": (ctypes.c_uint64, []),
     "mla_device_error_info": (None, [ctypes.POINTER(ctypes.c_uint32)]),
 }

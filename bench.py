@@ -471,7 +471,7 @@ ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
                   "bytes": (72_767_232 + 18_537_728) + (19_032_576 + 0),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
-                          "fac888e6957e39e953f1966007b9ff7fc03aa2ef3de6fd647d59beafc935e87a",
+                          "be48c633ee67393b190e64dbe7b47bc69163bb42f0b85349d5c10bdbae95315a",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
                           "8470448cc9cefd6bf7baa6b11f034bb548d5ccce3f5dfaf611570447dd93f53a"}}
 

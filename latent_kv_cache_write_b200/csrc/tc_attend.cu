@@ -1,4 +1,4 @@
-// Absorbed MLA attention on tcgen05 tensor cores (bf16, d_c = 512, d_R = 64).
+// Absorbed MLA attention on tcgen05 tensor cores (bf16, d_c = 512, d_R = 64 or 512).
 //
 // Rows of the problem are (query, head) pairs; all heads share the cached rows
 // [c_KV || k_R], which serve both as keys (all 576 dims) and as values (the 512 latent
@@ -6,8 +6,8 @@
 //
 // A 128 x 512 fp32 output accumulator fills a whole SM's tensor memory, so each 128-row
 // tile is handled by a cluster of two CTAs that split the latent dimension: CTA c owns
-// latent dims [256c, 256c + 256) and RoPE dims [32c, 32c + 32).  Per block of 64 keys
-// each CTA
+// latent dims [256c, 256c + 256) and half of the RoPE dims ([32c, 32c + 32) for d_R = 64,
+// [256c, 256c + 256) for d_R = 512).  Per block of 64 keys each CTA
 //   - TMA-loads its columns of the 64 cached rows (one load serves as K and as V),
 //   - computes its partial score S_c = Q_c . K_c^T with tcgen05.mma (Q's latent half
 //     resident in TMEM as the A operand, the RoPE part from shared memory),

@@ -615,6 +615,15 @@ def run_ours(args):
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl=wl)
+            # the same oracle on one thread (BLAS limited to one), a shorter sample
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    one = cpu_baseline(seconds=4.0, wl=wl)
+                line["cpu_baseline"]["single_thread"] = {"value": one["value"],
+                                                         "sample": one["sample"]}
+            except ImportError:
+                pass
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -108,8 +108,4 @@ __device__ __forceinline__ void rope_rotate_fast(float& a, float& b, double pos,
   b = nb;
 }
 
-__device__ __forceinline__ void set_device_error(unsigned int* err, unsigned int code) {
-  if (err) atomicOr(err, code);
-}
-
 }  // namespace mla

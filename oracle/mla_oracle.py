@@ -238,6 +238,50 @@ def attend_latent(q_abs: np.ndarray, cache: np.ndarray, q_first_tok: int,
     return o, lse
 
 
+def attend_latent_part(q_abs: np.ndarray, cache: np.ndarray, q_first_tok: int,
+                       k_first_tok: int, n_keys: int, scale: float, wl, key_lo: int,
+                       key_hi: int, queries: Optional[Iterable[Tuple[int, int]]] = None):
+    """One piece of a key range cut between workers: ``attend_latent`` over the visible keys
+    g with key_lo <= g < key_hi only (the cross-instance MLA abstract on the topic page
+    computes attention where the blocks live and merges the partial results).  Returns
+    (o_lat normalised over the piece, lse of the piece); a query without a visible key in
+    the piece gets o_lat = 0 and lse = -inf."""
+    q_abs = np.asarray(q_abs, dtype=np.float64)
+    cache = np.asarray(cache, dtype=np.float64)
+    d_c = wl.d_latent
+    sel = list(queries) if queries is not None else [
+        (b, i) for b in range(q_abs.shape[0]) for i in range(q_abs.shape[1])]
+    o = np.zeros((len(sel), q_abs.shape[2], d_c))
+    lse = np.full((len(sel), q_abs.shape[2]), -np.inf)
+    for n, (b, i) in enumerate(sel):
+        keys = visible_keys(q_first_tok + i, k_first_tok, n_keys, wl)
+        keys = keys[(keys >= key_lo) & (keys < key_hi)]
+        if keys.size == 0:
+            continue
+        rows = cache[b, keys % wl.ring_slots]
+        p, lse[n] = _softmax_lse(scale * (q_abs[b, i] @ rows.T))
+        o[n] = p @ rows[:, :d_c]
+    if queries is None:
+        B, T = q_abs.shape[0], q_abs.shape[1]
+        return o.reshape(B, T, *o.shape[1:]), lse.reshape(B, T, -1)
+    return o, lse
+
+
+def merge_partials(parts):
+    """Merge pieces (o_p, lse_p) of one softmax attention over disjoint key sets:
+    lse = log sum_p exp(lse_p) and o = sum_p exp(lse_p - lse) o_p (a piece with
+    lse_p = -inf has weight 0)."""
+    lses = np.stack([np.asarray(l, dtype=np.float64) for _, l in parts])      # [P, ...]
+    top = lses.max(axis=0)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    w = np.exp(lses - safe)                                                    # [P, ...]
+    tot = w.sum(axis=0)
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    o = sum(w[k][..., None] * np.asarray(op, dtype=np.float64) for k, (op, _) in enumerate(parts))
+    o = o / np.where(tot > 0, tot, 1.0)[..., None]
+    return o, lse
+
+
 def attend_materialised(q_nope: np.ndarray, q_rope: np.ndarray, cache: np.ndarray,
                         w_uk: np.ndarray, w_uv: np.ndarray, q_first_tok: int,
                         k_first_tok: int, n_keys: int, scale: float, wl,

@@ -384,6 +384,35 @@ def pin_ring_slots():
         assert np.array_equal(cache[:, s], O.cache_rows(h, w["w_dkv"], w["w_kr"], last, wl)[:, 0])
 
 
+def pin_split_key_merge():
+    """Attention over the visible keys cut into disjoint pieces at arbitrary points, each
+    piece normalised on its own and merged by log-sum-exp, equals the attention over all
+    of them; pieces past a query's last visible key carry no weight."""
+    for wl in (MINI, SMALL):
+        w, cache, qn, qr = build_state(wl, 0)
+        qa = O.absorb_q(qn, qr, w["w_uk"], wl.q_first_tok, wl)
+        full_o, full_l = O.attend_latent(qa, cache, wl.q_first_tok, wl.k_first_tok, wl.n_keys,
+                                         wl.softmax_scale, wl)
+        lo, hi = wl.k_first_tok, wl.k_first_tok + wl.n_keys
+        rng = np.random.default_rng(7)
+        for n_cut in (1, 2, 3):
+            cuts = sorted(set(rng.integers(lo + 1, hi, n_cut).tolist()))
+            edges = [lo] + cuts + [hi]
+            parts = [O.attend_latent_part(qa, cache, wl.q_first_tok, wl.k_first_tok, wl.n_keys,
+                                          wl.softmax_scale, wl, a, b)
+                     for a, b in zip(edges[:-1], edges[1:])]
+            o, l = O.merge_partials(parts)
+            assert rel(o, full_o) < 1e-12 and rel(l, full_l) < 1e-12, (wl.name, edges)
+        # the chunk's last frame as its own piece: earlier chunk frames see none of it
+        F = wl.tokens_per_frame
+        parts = [O.attend_latent_part(qa, cache, wl.q_first_tok, wl.k_first_tok, wl.n_keys,
+                                      wl.softmax_scale, wl, a, b)
+                 for a, b in ((lo, hi - F), (hi - F, hi))]
+        assert np.isneginf(parts[1][1][:, :F]).all()
+        o, l = O.merge_partials(parts)
+        assert rel(o, full_o) < 1e-12 and rel(l, full_l) < 1e-12
+
+
 def pin_frame_shift():
     """Re-indexing cached RoPE keys by whole frames equals writing the same hidden states
     at the shifted positions (rotations compose: R(p + d) = R(d) R(p), and a shift by
@@ -455,4 +484,5 @@ def pin_flop_counts():
 ALL_PINS = [pin_absorption_identity, pin_rope_relative, pin_rope_textbook_1d,
             pin_rope_axes, pin_rope_in_cache_and_query, pin_brute_force,
             pin_library_sdpa, pin_degenerate_cases, pin_mask_isolation,
-            pin_ring_slots, pin_frame_shift, pin_cache_bytes, pin_flop_counts]
+            pin_ring_slots, pin_split_key_merge, pin_frame_shift, pin_cache_bytes,
+            pin_flop_counts]

@@ -10,7 +10,7 @@ from tests import oracle_pins as P
 _orig = {n: getattr(O, n) for n in (
     "rotate_pairs", "rope_angles", "token_position", "visible_keys", "attend_latent",
     "attend_materialised", "absorb_q", "ring_slot", "up_v", "cache_rows", "_softmax_lse",
-    "mla_bytes_per_token", "rope3d", "shift_frames")}
+    "mla_bytes_per_token", "rope3d", "shift_frames", "merge_partials")}
 
 
 def _rot_sign(v, angles):
@@ -86,6 +86,18 @@ def _bytes_no_rope(d_latent, d_rope, elem_bytes):
     return d_latent * elem_bytes
 
 
+def _merge_unweighted(parts):
+    # the plain mean of the pieces, ignoring how much of the softmax mass each holds
+    o = sum(np.asarray(op, dtype=np.float64) for op, _ in parts) / len(parts)
+    return o, _orig["merge_partials"](parts)[1]
+
+
+def _merge_lse_max(parts):
+    # the largest piece's log-sum-exp instead of the log of the summed masses
+    o, _ = _orig["merge_partials"](parts)
+    return o, np.max(np.stack([l for _, l in parts]), axis=0)
+
+
 def _shift_row_axis(cache, first_tok, n_tok, delta_frames, wl):
     # turns the y pairs instead of the t pairs
     out = np.array(cache, dtype=np.float64, copy=True)
@@ -117,6 +129,8 @@ MUTATIONS = {
     "cache_bytes_drop_rope": ("mla_bytes_per_token", _bytes_no_rope),
     "shift_turns_row_axis": ("shift_frames", _shift_row_axis),
     "shift_backwards": ("shift_frames", _shift_backwards),
+    "merge_unweighted": ("merge_partials", _merge_unweighted),
+    "merge_lse_max": ("merge_partials", _merge_lse_max),
 }
 
 

@@ -466,14 +466,19 @@ def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
 # DRAM bytes (read + write) of one chunk mla_attend call, from the ncu captures summarised in
 # profiles/attend_kernel_video_chunk.md (the attention kernel) and
 # profiles/combine_kernel_video_chunk.md (the split-key merge).  Counters describe the kernel
-# sources they were taken on: the value is reported only while those sources are unchanged.
+# sources they were taken on (the two kernels and the headers they compile in): the value is
+# reported only while those sources are unchanged.
 ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
-                  "bytes": (72_767_232 + 18_537_728) + (19_032_576 + 0),
+                  "bytes": (72_785_152 + 18_896_384) + (19_032_576 + 0),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
-                          "be48c633ee67393b190e64dbe7b47bc69163bb42f0b85349d5c10bdbae95315a",
+                          "7610bd26aa018ef493220a9d67f1578810d74b107ff0d9b3c5502f8369d1b233",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
-                          "8470448cc9cefd6bf7baa6b11f034bb548d5ccce3f5dfaf611570447dd93f53a"}}
+                          "8470448cc9cefd6bf7baa6b11f034bb548d5ccce3f5dfaf611570447dd93f53a",
+                      "latent_kv_cache_write_b200/csrc/attend_common.cuh":
+                          "7c6b9296fbd5887b502af791bfe503be8bdd583aa91ba619787cfd443f03611b",
+                      "latent_kv_cache_write_b200/csrc/tc_ptx.cuh":
+                          "acf340a739dda6050cfa0f506bb620cde4db63bf01d97690f8aae4305ee2c25d"}}
 
 
 def attend_traffic(wl=WORKLOAD):

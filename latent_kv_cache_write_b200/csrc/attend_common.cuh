@@ -22,6 +22,7 @@ struct AttnArgs {
   float* ws_lse;            // their natural log-sum-exps, one per CTA half [slot][2][TM]
   int tiles_per_batch;
   int bn;                   // keys per block of the launch
+  int pf;                   // L2 look-ahead of the key loads in blocks (0: none)
   unsigned int* err;
 };
 

@@ -111,6 +111,7 @@ struct Lay {
 };
 
 constexpr uint32_t O_COL = 0, Q_COL = 256, S_COL = 384;
+constexpr int PF_BLOCKS = 1;                  // L2 look-ahead of the key loads (decode)
 constexpr unsigned FULL = 0xffffffffu;
 
 // Cluster c walks the key blocks from (cut_tile[c], cut_blk[c]) up to, not including,
@@ -269,9 +270,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmKR);
+      // With a.pf > 0 the boxes of block j + a.pf are asked into L2 while block j's stage
+      // is awaited: keys that no other tile reads come from HBM, and a stage is held from
+      // its load to its PV product, so the stages alone keep too few loads in flight.
+      auto prefetch_block = [&](int j) {
+        int64_t slot0, g0;
+        int valid;
+        sw.tg.blk.get(j, slot0, g0, valid);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tma_prefetch_l2_3d(&tmK, (int)rank * HALF + q * 64, (int32_t)slot0, sw.tg.b);
+        if constexpr (LY::WIDE) {
+#pragma unroll
+          for (int q = 0; q < LY::NRB; ++q)
+            tma_prefetch_l2_3d(&tmK, G.Dc + (int)rank * LY::RHALF + q * 64, (int32_t)slot0,
+                               sw.tg.b);
+        } else {
+          tma_prefetch_l2_3d(&tmKR, G.Dc + (int)rank * LY::RHALF, (int32_t)slot0, sw.tg.b);
+        }
+      };
       bool ok = true;
       for (; ok && sw.valid(); sw.next(a)) {
+        if (a.pf > 0)
+          for (int j = sw.jb; j < sw.je && j < sw.jb + a.pf; ++j) prefetch_block(j);
         for (int j = sw.jb; j < sw.je; ++j) {
+          if (a.pf > 0 && j + a.pf < sw.je) prefetch_block(j + a.pf);
           const int g = sw.gbase + (j - sw.jb);
           const int s = g % NST;
           const uint32_t fph = ((g / NST) & 1) ^ 1;
@@ -802,6 +825,9 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.lse = lse;
   a.tiles_per_batch = tiles_per_batch;
   a.bn = bn;
+  // a sequence's keys are read by its tiles only: with one or two tiles (decode) each key
+  // block comes from HBM once, and the producer looks PF_BLOCKS blocks ahead
+  a.pf = tiles_per_batch <= 2 ? PF_BLOCKS : 0;
   a.err = err;
   const bool split = workspace != nullptr && workspace_bytes >= tc_attend_workspace(g);
 

@@ -381,6 +381,47 @@ def shift_leg(torch, mla, step, steps, warmup, flush):
                     "launch-bound"}
 
 
+def quant_token_bytes(wl, content_bits: int, rope_bits: int) -> int:
+    """Bytes of one token in the low-bit ring: both packed paths and two float32 scales."""
+    return wl.d_latent * content_bits // 8 + wl.d_rope * rope_bits // 8 + 8
+
+
+def quant_leg(torch, mla, step, steps, warmup, flush, bits=(4, 4)):
+    """The window's rows into the low-bit ring (mla_cache_quantise), and back into a second
+    ring (mla_cache_dequantise); INT4 content and RoPE by default."""
+    wl = step.wl
+    cb, rb = bits
+    B, S, n = wl.batch, wl.ring_slots, wl.n_keys
+    qc = torch.empty((B, S, wl.d_latent * cb // 8), dtype=torch.uint8, device="cuda")
+    qr = torch.empty((B, S, wl.d_rope * rb // 8), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((B, S), dtype=torch.float32, device="cuda")
+    sr = torch.empty_like(sc)
+    back = torch.empty_like(step.cache)
+
+    def quant(_a=None):
+        mla.mla_cache_quantise(step.shape, step.cache, wl.k_first_tok, n, cb, rb, qc, qr, sc,
+                               sr)
+
+    def dequant(_a=None):
+        mla.mla_cache_dequantise(step.shape, qc, qr, sc, sr, cb, rb, wl.k_first_tok, n, back)
+
+    for _ in range(warmup):
+        quant()
+        dequant()
+    ms_q, _ = time_steps(torch, quant, steps, flush)
+    ms_d, _ = time_steps(torch, dequant, steps, flush)
+    row = wl.row_width * wl.elem_bytes
+    packed = quant_token_bytes(wl, cb, rb)
+    moved = B * n * (row + packed)                    # one side read, the other written
+    tq, td = statistics.mean(ms_q), statistics.mean(ms_d)
+    return {"calls": "mla_cache_quantise, mla_cache_dequantise",
+            "bits": {"content": cb, "rope": rb}, "rows": B * n, "bytes_per_token": packed,
+            "compression": row / packed, "bytes": moved,
+            "quantise": {"ms": tq, "value": moved / (tq * 1e-3) / 1e9, "unit": "GB/s"},
+            "dequantise": {"ms": td, "value": moved / (td * 1e-3) / 1e9, "unit": "GB/s"},
+            "note": "the window's rows; ~9 MB each way, so launch- and latency-bound"}
+
+
 def decode_leg(torch, mla, steps, warmup, flush, wl=C.DECODE):
     shape = mla.make_shape(wl)
     dev = "cuda"
@@ -574,6 +615,8 @@ def run_ours(args):
         mat["frac"] = mat["tflops"] / float(peaks["bf16_tflops"])
     shift = shift_leg(torch, mla, step, max(3, args.steps), args.warmup, flush) \
         if rank == 0 else None
+    quant = quant_leg(torch, mla, step, max(3, args.steps), args.warmup, flush) \
+        if rank == 0 else None
     if dec:
         dec["peak_gbs"] = float(peaks["hbm_gbs"])
         dec["frac"] = dec["value"] / dec["peak_gbs"]
@@ -615,6 +658,7 @@ def run_ours(args):
             "decode": dec,
             "materialised": mat,
             "k_rope_shift": shift,
+            "quant_ring": quant,
             "clocks": clocks.summary(),
             "kernels_ms": kernels_ms,
         }

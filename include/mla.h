@@ -228,6 +228,50 @@ mla_status mla_cache_shift_frames(const mla_shape* shape, void* cache, int64_t f
                                   int64_t n_tok, int64_t delta_frames, void* stream);
 
 /*
+ * mla_cache_quantise — the low-bit latent ring (QuantMLA abstract on the "Multi-Head Latent
+ * Attention" topic page: the content latent and the RoPE key are cached at low bit width,
+ * INT4 and INT4, or INT2 content with an INT4 RoPE key, each path with a quantiser of its
+ * own).  The path's learned transformations are not applied: each path of each row has one
+ * scale.
+ *
+ * For b < B and the slots r = g mod S of g = first_tok .. first_tok + n_tok - 1, the content
+ * part x = cache[b][r][0 : d_latent] (and likewise the RoPE part cache[b][r][d_latent :]) is
+ * quantised with q = 2^(bits-1) - 1:
+ *   scale[b][r] = max|x| / q                              (float32, correctly rounded)
+ *   code_i = x_i / scale rounded to the nearest integer (ties to even; float32 division),
+ *            clipped to [-q, q]                           (all 0 when the scale is 0)
+ * and the codes are stored as two's-complement fields of `bits` bits, little-endian: code i
+ * at bits [i*bits, (i+1)*bits) of the packed row, byte k holding bits [8k, 8k + 8).
+ *
+ *   cache     [B, S, d_latent + d_rope]          read at n_tok slots (finite values)
+ *   q_content [B, S, d_latent * content_bits / 8] bytes, written at those slots
+ *   q_rope    [B, S, d_rope * rope_bits / 8]      bytes, written at those slots
+ *   scale_c, scale_r [B, S] float32               written at those slots
+ * content_bits and rope_bits are 2, 4 or 8.  Other slots are not touched.
+ * Errors: MLA_ERR_ARG for a NULL pointer, n_tok < 0 or a bit width other than 2, 4, 8;
+ * MLA_ERR_UNSUPPORTED unless d_latent and d_rope are multiples of 8 and at most 1024;
+ * MLA_ERR_RANGE if n_tok > S or first_tok < 0; MLA_ERR_ALIGN for a pointer not 16-byte
+ * aligned.
+ */
+mla_status mla_cache_quantise(const mla_shape* shape, const void* cache, int64_t first_tok,
+                              int64_t n_tok, int32_t content_bits, int32_t rope_bits,
+                              void* q_content, void* q_rope, float* scale_c, float* scale_r,
+                              void* stream);
+
+/*
+ * mla_cache_dequantise — the rows a low-bit ring stands for (the inverse of
+ * mla_cache_quantise): for the same slots,
+ *   cache[b][r][i] = code_i * scale[b][r]   (the float32 product, rounded to the storage
+ *                                            dtype to nearest even)
+ * for both paths.  Arguments as in mla_cache_quantise, with the packed ring and scales read
+ * and the cache written at n_tok slots; the same errors.
+ */
+mla_status mla_cache_dequantise(const mla_shape* shape, const void* q_content,
+                                const void* q_rope, const float* scale_c,
+                                const float* scale_r, int32_t content_bits, int32_t rope_bits,
+                                int64_t first_tok, int64_t n_tok, void* cache, void* stream);
+
+/*
  * mla_attend_materialised_workspace_size — bytes of device workspace mla_attend_materialised
  * needs: the per-head keys and then the per-head values of every ring slot, bf16,
  * 2 * B * S * n_h * d_nope * 2 bytes.  0 for shapes the call does not support.

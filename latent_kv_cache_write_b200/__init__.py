@@ -16,6 +16,7 @@ from .native import MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
            "mla_attend_fixed_scratch", "mla_attend_materialised", "mla_cache_shift_frames",
+           "mla_cache_quantise", "mla_cache_dequantise",
            "mla_attend_materialised_workspace_size", "mla_up_v", "mla_device_error",
            "mla_kernel_launches", "mla_device_error_info", "mla_check_wait_timeout", "make_shape",
            "MlaShape", "MlaError"]
@@ -80,6 +81,22 @@ def mla_cache_shift_frames(shape: MlaShape, cache, first_tok: int, n_tok: int,
                            delta_frames: int, stream=None) -> None:
     native.check("mla_cache_shift_frames", native.lib().mla_cache_shift_frames(
         ctypes.byref(shape), _ptr(cache), first_tok, n_tok, delta_frames, _stream(stream)))
+
+
+def mla_cache_quantise(shape: MlaShape, cache, first_tok: int, n_tok: int, content_bits: int,
+                       rope_bits: int, q_content, q_rope, scale_c, scale_r,
+                       stream=None) -> None:
+    native.check("mla_cache_quantise", native.lib().mla_cache_quantise(
+        ctypes.byref(shape), _ptr(cache), first_tok, n_tok, content_bits, rope_bits,
+        _ptr(q_content), _ptr(q_rope), _ptr(scale_c), _ptr(scale_r), _stream(stream)))
+
+
+def mla_cache_dequantise(shape: MlaShape, q_content, q_rope, scale_c, scale_r,
+                         content_bits: int, rope_bits: int, first_tok: int, n_tok: int, cache,
+                         stream=None) -> None:
+    native.check("mla_cache_dequantise", native.lib().mla_cache_dequantise(
+        ctypes.byref(shape), _ptr(q_content), _ptr(q_rope), _ptr(scale_c), _ptr(scale_r),
+        content_bits, rope_bits, first_tok, n_tok, _ptr(cache), _stream(stream)))
 
 
 def mla_attend_materialised_workspace_size(shape: MlaShape) -> int:

@@ -45,6 +45,17 @@ cudaError_t tc_materialise(const Geo& g, const void* cache, const void* w, void*
 cudaError_t shift_frames(const Geo& g, bool bf, void* cache, int64_t first_tok, int64_t n_tok,
                          int64_t delta_frames, cudaStream_t st);
 
+// Low-bit latent ring (quant.cu): per-row, per-path scale quantisation of the ring rows of
+// tokens first_tok .. first_tok + n_tok - 1 into packed codes and float32 scales, and the
+// inverse.  quant_supported: both paths a multiple of 8 and at most 1024 wide.
+bool quant_supported(const Geo& g);
+cudaError_t quantise_ring(const Geo& g, bool bf, const void* cache, int64_t first_tok,
+                          int64_t n_tok, int cbits, int rbits, void* qc, void* qr, float* sc,
+                          float* sr, cudaStream_t st);
+cudaError_t dequantise_ring(const Geo& g, bool bf, const void* qc, const void* qr,
+                            const float* sc, const float* sr, int cbits, int rbits,
+                            int64_t first_tok, int64_t n_tok, void* cache, cudaStream_t st);
+
 // Non-absorbed attention over the materialised keys and values (tc_attend_mat.cu).
 bool tc_attend_mat_supported(const Geo& g);
 cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,

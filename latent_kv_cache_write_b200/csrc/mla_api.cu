@@ -65,6 +65,26 @@ mla_status cuda_status(cudaError_t e) {
   return MLA_ERR_CUDA;
 }
 
+
+bool quant_bits_ok(int32_t b) { return b == 2 || b == 4 || b == 8; }
+
+// the checks both directions of the low-bit ring share
+mla_status check_quant(const mla_shape* shape, Geo* g, int64_t first_tok, int64_t n_tok,
+                       int32_t cbits, int32_t rbits, const void* cache, const void* qc,
+                       const void* qr, const float* sc, const float* sr) {
+  mla_status st = check_shape(shape, g);
+  if (st != MLA_OK) return st;
+  if (!cache || !qc || !qr || !sc || !sr || n_tok < 0 || !quant_bits_ok(cbits) ||
+      !quant_bits_ok(rbits))
+    return MLA_ERR_ARG;
+  if (!quant_supported(*g)) return MLA_ERR_UNSUPPORTED;
+  if (first_tok < 0 || n_tok > g->S) return MLA_ERR_RANGE;
+  if (!aligned16(cache) || !aligned16(qc) || !aligned16(qr) || !aligned16(sc) ||
+      !aligned16(sr))
+    return MLA_ERR_ALIGN;
+  return MLA_OK;
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -216,6 +236,34 @@ mla_status mla_cache_shift_frames(const mla_shape* shape, void* cache, int64_t f
   if (n_tok == 0) return MLA_OK;
   return cuda_status(shift_frames(g, shape->dtype == MLA_BF16, cache, first_tok, n_tok,
                                   delta_frames, (cudaStream_t)stream));
+}
+
+mla_status mla_cache_quantise(const mla_shape* shape, const void* cache, int64_t first_tok,
+                              int64_t n_tok, int32_t content_bits, int32_t rope_bits,
+                              void* q_content, void* q_rope, float* scale_c, float* scale_r,
+                              void* stream) {
+  Geo g;
+  mla_status st = check_quant(shape, &g, first_tok, n_tok, content_bits, rope_bits, cache,
+                              q_content, q_rope, scale_c, scale_r);
+  if (st != MLA_OK) return st;
+  if (n_tok == 0) return MLA_OK;
+  return cuda_status(quantise_ring(g, shape->dtype == MLA_BF16, cache, first_tok, n_tok,
+                                   content_bits, rope_bits, q_content, q_rope, scale_c,
+                                   scale_r, (cudaStream_t)stream));
+}
+
+mla_status mla_cache_dequantise(const mla_shape* shape, const void* q_content,
+                                const void* q_rope, const float* scale_c,
+                                const float* scale_r, int32_t content_bits, int32_t rope_bits,
+                                int64_t first_tok, int64_t n_tok, void* cache, void* stream) {
+  Geo g;
+  mla_status st = check_quant(shape, &g, first_tok, n_tok, content_bits, rope_bits, cache,
+                              q_content, q_rope, scale_c, scale_r);
+  if (st != MLA_OK) return st;
+  if (n_tok == 0) return MLA_OK;
+  return cuda_status(dequantise_ring(g, shape->dtype == MLA_BF16, q_content, q_rope, scale_c,
+                                     scale_r, content_bits, rope_bits, first_tok, n_tok, cache,
+                                     (cudaStream_t)stream));
 }
 
 size_t mla_attend_materialised_workspace_size(const mla_shape* shape) {

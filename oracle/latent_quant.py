@@ -124,12 +124,14 @@ def empty_quant_cache(wl, content_bits: int, rope_bits: int) -> Dict[str, np.nda
     }
 
 
-def quantise_row_paths(rows: np.ndarray, wl, content_bits: int, rope_bits: int):
-    """(packed content, packed rope, scale_c, scale_r) of cached rows [..., d_c + d_R]."""
+def quantise_row_paths(rows: np.ndarray, wl, content_bits: int, rope_bits: int,
+                       decide=np.float64):
+    """(packed content, packed rope, scale_c, scale_r) of cached rows [..., d_c + d_R];
+    ``decide`` as in quantise_rows."""
     rows = np.asarray(rows, dtype=np.float64)
     d_c = wl.d_latent
-    cc, sc = quantise_rows(rows[..., :d_c], content_bits)
-    cr, sr = quantise_rows(rows[..., d_c:], rope_bits)
+    cc, sc = quantise_rows(rows[..., :d_c], content_bits, decide)
+    cr, sr = quantise_rows(rows[..., d_c:], rope_bits, decide)
     return pack_codes(cc, content_bits), pack_codes(cr, rope_bits), sc, sr
 
 

@@ -176,3 +176,32 @@ def test_shift_frames_validation(L):
     assert sh(first=-1) == native.MLA_ERR_RANGE
     assert sh(cache=ODD) == native.MLA_ERR_ALIGN
     assert sh(n=0) == native.MLA_OK                             # empty: nothing to do
+
+
+def test_quantise_validation(L):
+    s = _shape()
+    f32 = _shape(dtype=native.MLA_F32)
+
+    def q(fn="mla_cache_quantise", shape=s, **k):
+        ptrs = [k.get("cache", FAKE), k.get("qc", FAKE), k.get("qr", FAKE), k.get("sc", FAKE),
+                k.get("sr", FAKE)]
+        first, n, cb, rb = k.get("first", 0), k.get("n", 6240), k.get("cb", 4), k.get("rb", 4)
+        if fn == "mla_cache_quantise":
+            return L.mla_cache_quantise(ctypes.byref(shape), ptrs[0], first, n, cb, rb, *ptrs[1:],
+                                        None)
+        return L.mla_cache_dequantise(ctypes.byref(shape), ptrs[1], ptrs[2], ptrs[3], ptrs[4],
+                                      cb, rb, first, n, ptrs[0], None)
+
+    for fn in ("mla_cache_quantise", "mla_cache_dequantise"):
+        for name in ("cache", "qc", "qr", "sc", "sr"):
+            assert q(fn, **{name: None}) == native.MLA_ERR_ARG, (fn, name)
+            assert q(fn, **{name: ODD}) == native.MLA_ERR_ALIGN, (fn, name)
+        assert q(fn, n=-1) == native.MLA_ERR_ARG
+        for bad in (0, 1, 3, 5, 16):
+            assert q(fn, cb=bad) == native.MLA_ERR_ARG and q(fn, rb=bad) == native.MLA_ERR_ARG
+        assert q(fn, n=6241) == native.MLA_ERR_RANGE
+        assert q(fn, first=-1) == native.MLA_ERR_RANGE
+        assert q(fn, shape=_shape(d_latent=516)) == native.MLA_ERR_UNSUPPORTED
+        assert q(fn, shape=_shape(d_latent=2048)) == native.MLA_ERR_UNSUPPORTED
+        assert q(fn, n=0) == native.MLA_OK
+        assert q(fn, shape=f32, n=0, cb=2, rb=8) == native.MLA_OK

@@ -62,3 +62,11 @@ def test_percentiles_nearest_rank():
 def test_step_workloads():
     assert bench.STEP_WORKLOADS == ("video_chunk_bf16", "long_window_bf16", "wide_key_bf16")
     assert bench.WORKLOAD.name == "video_chunk_bf16"
+
+
+def test_quant_ring_bytes():
+    wl = C.VIDEO_CHUNK
+    # INT4 content (256 B) and RoPE (32 B) plus two float32 scales, against 1152 B in bf16
+    assert bench.quant_token_bytes(wl, 4, 4) == 296
+    assert bench.quant_token_bytes(wl, 2, 4) == 168
+    assert bench.quant_token_bytes(C.WIDE_KEY, 4, 4) == 256 + 256 + 8

@@ -61,7 +61,7 @@ def _unpack_unsigned(packed, bits, n):
     return (c & ((1 << bits) - 1)).astype(np.int8)
 
 
-def _shared_scale(rows, wl, cb, rb):
+def _shared_scale(rows, wl, cb, rb, decide=np.float64):
     # one scale over the whole row, both paths
     rows = np.asarray(rows, dtype=np.float64)
     d_c = wl.d_latent

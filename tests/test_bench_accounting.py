@@ -70,3 +70,11 @@ def test_quant_ring_bytes():
     assert bench.quant_token_bytes(wl, 4, 4) == 296
     assert bench.quant_token_bytes(wl, 2, 4) == 168
     assert bench.quant_token_bytes(C.WIDE_KEY, 4, 4) == 256 + 256 + 8
+
+
+def test_both_arms_report_one_config():
+    wl = C.VIDEO_CHUNK
+    cfg = bench.step_config(wl, 2)
+    assert cfg["workload"] == wl.name and cfg["keys"] == 6240 and cfg["queries"] == 1560
+    assert cfg["flops_per_step"] == sum(bench.step_flops(wl).values())
+    assert cfg["parallelism"] == "replicas x2 (independent sequences)"

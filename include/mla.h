@@ -35,6 +35,9 @@
  *     elements; pair j of an axis segment with n pairs, elements (2j, 2j+1) of the
  *     segment, is rotated by pos_a * rope_theta^(-j/n) radians.
  *   - Accumulation is float32.  bfloat16 results are rounded to nearest even.
+ *   - Sizes: batch * ring_slots, and for the calls that take queries
+ *     batch * n_q * n_heads, are at most 2^31 - 1 (rows are addressed with 32-bit
+ *     tensor coordinates); larger shapes return MLA_ERR_UNSUPPORTED.
  */
 #ifndef MLA_H
 #define MLA_H

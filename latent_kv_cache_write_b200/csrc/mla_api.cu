@@ -49,6 +49,8 @@ mla_status check_shape(const mla_shape* s, Geo* g) {
   if (s->dtype != MLA_F32 && s->dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
   if ((int64_t)s->d_latent + s->d_rope > 32 * 40) return MLA_ERR_UNSUPPORTED;
   if ((int64_t)s->batch * s->n_heads > 65535) return MLA_ERR_UNSUPPORTED;
+  // ring rows are addressed with 32-bit tensor coordinates
+  if ((int64_t)s->batch * s->ring_slots > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   g->B = s->batch; g->H = s->n_heads; g->Dn = s->d_nope; g->Dc = s->d_latent; g->Dr = s->d_rope;
   for (int i = 0; i < 3; ++i) g->pairs[i] = s->rope_pairs[i];
   g->theta = s->rope_theta;
@@ -136,7 +138,7 @@ mla_status mla_absorb_q(const mla_shape* shape, const void* q_nope, const void* 
   if (st != MLA_OK) return st;
   if (n_q < 0 || !q_nope || !w_uk || !q_abs || (g.Dr > 0 && !q_rope)) return MLA_ERR_ARG;
   if (q_first_tok < 0) return MLA_ERR_RANGE;
-  if (n_q > INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  if (n_q > INT32_MAX / 2 || (int64_t)g.B * n_q * g.H > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   if (!aligned16(q_nope) || (q_rope && !aligned16(q_rope)) || !aligned16(w_uk) ||
       !aligned16(q_abs))
     return MLA_ERR_ALIGN;
@@ -169,7 +171,7 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
   if (n_keys < 1 || n_keys > g.S || k_first_tok < 0 || q_first_tok < k_first_tok ||
       q_first_tok + n_q > k_first_tok + n_keys)
     return MLA_ERR_RANGE;
-  if (n_q > 65535) return MLA_ERR_UNSUPPORTED;
+  if (n_q > 65535 || (int64_t)g.B * n_q * g.H > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(o_lat) || (lse && !aligned16(lse)))
     return MLA_ERR_ALIGN;
   // no workspace at all is allowed (the schedule then keeps tiles whole); a workspace
@@ -215,7 +217,7 @@ mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, cons
   mla_status st = check_shape(shape, &g);
   if (st != MLA_OK) return st;
   if (n_q < 0 || !o_lat || !w_uv || !out) return MLA_ERR_ARG;
-  if (n_q > INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  if (n_q > INT32_MAX / 2 || (int64_t)g.B * n_q * g.H > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   if (!aligned16(o_lat) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_ALIGN;
   if (n_q == 0) return MLA_OK;
   const bool bf = shape->dtype == MLA_BF16;
@@ -289,7 +291,8 @@ mla_status mla_attend_materialised(const mla_shape* shape, const void* q_nope,
       q_first_tok + n_q > k_first_tok + n_keys)
     return MLA_ERR_RANGE;
   const size_t need = mla_attend_materialised_workspace_size(shape);
-  if (need == 0 || n_q > 65535) return MLA_ERR_UNSUPPORTED;
+  if (need == 0 || n_q > 65535 || (int64_t)g.B * n_q * g.H > INT32_MAX)
+    return MLA_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < need) return MLA_ERR_ARG;
   if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(cache) || !aligned16(w_uk) ||
       !aligned16(w_uv) || !aligned16(out) || (lse && !aligned16(lse)) || !aligned16(workspace))

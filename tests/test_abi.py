@@ -205,3 +205,23 @@ def test_quantise_validation(L):
         assert q(fn, shape=_shape(d_latent=2048)) == native.MLA_ERR_UNSUPPORTED
         assert q(fn, n=0) == native.MLA_OK
         assert q(fn, shape=f32, n=0, cb=2, rb=8) == native.MLA_OK
+
+
+def test_row_counts_beyond_32_bit_coordinates(L):
+    U = native.MLA_ERR_UNSUPPORTED
+    # batch x ring_slots rows: refused by every call, before anything else is looked at
+    huge_ring = _shape(ring_slots=1 << 31)
+    assert _attend(L, huge_ring) == U
+    assert L.mla_cache_shift_frames(ctypes.byref(huge_ring), FAKE, 0, 1, 1, None) == U
+    assert L.mla_cache_quantise(ctypes.byref(_shape(batch=2, ring_slots=1 << 30)), FAKE, 0, 1,
+                                4, 4, FAKE, FAKE, FAKE, FAKE, None) == U
+    assert L.mla_attend_workspace_size(ctypes.byref(huge_ring), 1, 1) == 0
+    # batch x n_q x n_heads query rows
+    s = _shape(batch=2, n_heads=32)
+    n = 1 << 25                                           # 2 x 2^25 x 32 = 2^31 rows
+    assert L.mla_absorb_q(ctypes.byref(s), FAKE, FAKE, n, 0, FAKE, FAKE, None) == U
+    assert L.mla_up_v(ctypes.byref(s), FAKE, n, FAKE, FAKE, None) == U
+    assert L.mla_absorb_q(ctypes.byref(s), FAKE, FAKE, 0, 0, FAKE, FAKE, None) == native.MLA_OK
+    big = _shape(batch=1000, n_heads=65, ring_slots=50000)    # 1000 x 40000 x 65 rows
+    assert _attend(L, big, n_q=40000, q_first=0, n_keys=50000) == U
+    assert _mat(L, big, n_q=40000, q_first=0, n_keys=50000, ws_bytes=1 << 62) == U

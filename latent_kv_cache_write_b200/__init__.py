@@ -4,6 +4,25 @@ Python face of ``libmla.so``: the calls of the C ABI under the same names, takin
 ``torch`` CUDA tensors (or raw device pointers) and enqueuing on the current CUDA
 stream unless a stream is given.  PyTorch supplies device memory and streams only;
 all arithmetic runs in the library's kernels.
+
+One chunk step (bf16; B sequences, T new tokens of one frame written at token g0, the
+chunk's queries attending to the n_keys window tokens starting at k0)::
+
+    import latent_kv_cache_write_b200 as mla
+    shape = mla.MlaShape(batch=B, n_heads=H, d_nope=128, d_latent=512, d_rope=64,
+                         rope_pairs=(8, 12, 12), rope_theta=1e4, grid_h=gh, grid_w=gw,
+                         ring_slots=S, dtype=mla.native.MLA_BF16)
+    mla.mla_cache_write(shape, h, d_model, T, g0, w_dkv, w_kr, cache)   # ring [B, S, 576]
+    mla.mla_absorb_q(shape, q_nope, q_rope, T, g0, w_uk, q_abs)          # [B, T, H, 576]
+    ws = torch.empty(mla.mla_attend_workspace_size(shape, T, n_keys), dtype=torch.uint8,
+                     device="cuda")
+    mla.mla_attend(shape, q_abs, T, g0, cache, k0, n_keys, scale, o_lat, lse, ws)
+    mla.mla_up_v(shape, o_lat, T, w_uv, out)                             # [B, T, H, 128]
+
+``mla_attend_materialised`` replaces the last three calls with the non-absorbed form;
+``mla_cache_shift_frames`` re-indexes the window's RoPE keys by whole frames;
+``mla_cache_quantise`` / ``mla_cache_dequantise`` convert ring rows to and from the
+low-bit ring.  Errors raise ``MlaError`` with the library's status.
 """
 
 from __future__ import annotations

@@ -55,19 +55,9 @@ def token_position(g: int, grid_h: int, grid_w: int) -> Tuple[int, int, int]:
     return g // f, (g % f) // grid_w, g % grid_w
 
 
-def frame_of(g: int, grid_h: int, grid_w: int) -> int:
-    return g // (grid_h * grid_w)
-
-
 def ring_slot(g: int, ring_slots: int) -> int:
     """Slot of global token g in a sliding-window ring of ``ring_slots`` tokens."""
     return g % ring_slots
-
-
-def key_visible(g_query: int, g_key: int, grid_h: int, grid_w: int) -> bool:
-    """Frame-block-causal visibility: a query sees every key of its own and earlier
-    frames (next-frame prediction over a sliding window, [VideoMLA] "The Gap")."""
-    return frame_of(g_key, grid_h, grid_w) <= frame_of(g_query, grid_h, grid_w)
 
 
 # ----------------------------------------------------------------------------------
@@ -196,7 +186,9 @@ def absorb_q(q_nope: np.ndarray, q_rope: np.ndarray, w_uk: np.ndarray, q_first_t
 
 
 def visible_keys(g_query: int, k_first_tok: int, n_keys: int, wl) -> np.ndarray:
-    """Global tokens of the window that query g_query may attend to."""
+    """Global tokens of the window that query g_query may attend to: frame-block-causal,
+    every key of its own and earlier frames (next-frame prediction over a sliding
+    window, [VideoMLA] "The Gap")."""
     ks = np.arange(k_first_tok, k_first_tok + n_keys, dtype=np.int64)
     f = wl.grid_h * wl.grid_w
     return ks[ks // f <= g_query // f]

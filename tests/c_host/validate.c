@@ -34,5 +34,13 @@ int main(void) {
   /* empty calls succeed without touching the device */
   printf("empty_up_v %s\n", mla_status_string(mla_up_v(&s, fake, 0, fake, fake, NULL)));
   printf("empty_shift %s\n", mla_status_string(mla_cache_shift_frames(&s, fake, 0, 0, 1, NULL)));
+  /* the low-bit ring: a 3-bit code width is refused, an empty range succeeds */
+  float* fs = (float*)(void*)fake;
+  printf("quant_bits %s\n",
+         mla_status_string(mla_cache_quantise(&s, fake, 0, 6240, 3, 4, fake, fake, fs, fs,
+                                              NULL)));
+  printf("empty_dequant %s\n",
+         mla_status_string(mla_cache_dequantise(&s, fake, fake, fs, fs, 2, 4, 0, 0, fake,
+                                                NULL)));
   return 0;
 }

@@ -23,11 +23,13 @@ def test_plain_c_host(tmp_path):
                    check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True,
                          timeout=120).stdout.split("\n")
-    assert out[:6] == [
+    assert out[:8] == [
         "status MLA_ERR_RANGE",
         f"materialised_ws {2 * 6240 * 32 * 128 * 2}",
         "attend_range MLA_ERR_RANGE",
         "shape_arg MLA_ERR_ARG",
         "empty_up_v MLA_OK",
         "empty_shift MLA_OK",
+        "quant_bits MLA_ERR_ARG",
+        "empty_dequant MLA_OK",
     ]

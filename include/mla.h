@@ -152,6 +152,12 @@ size_t mla_attend_workspace_size(const mla_shape* shape, int64_t n_q, int64_t n_
  *   are few tiles or they do not divide evenly).  Calls that share a workspace must
  *   not run concurrently.
  * A single query per sequence (n_q == 1) is the decode case.
+ * Score range: any inputs whose scores are finite in float32.  The bfloat16 tensor-core
+ * path splits each score's dot product between two SMs and sums the two partials; a
+ * partial whose magnitude times softmax_scale * log2(e) is at most 8 is passed on rounded
+ * to fp16 (an error of at most 2^-8 in the exponent's log2 units, a fraction of a percent
+ * of a softmax weight, like the bf16 rounding of P); larger partials, up to the float32
+ * range, are passed on exactly, at the cost of two more exchanges for the key block.
  * Errors: MLA_ERR_RANGE if n_keys > S, n_keys < 1, or the queries are not inside the
  * key window (k_first_tok <= q_first_tok and q_first_tok + n_q <= k_first_tok +
  * n_keys); MLA_ERR_ARG if a workspace is given (or workspace_bytes > 0) and it is
@@ -182,7 +188,10 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
  *     than MLA_FIXED_SCRATCH_BYTES (mla_attend_workspace_size() > it);
  *   - MLA_ERR_CUDA if the array's device address cannot be obtained.
  * The first call on a device looks the array's address up (cudaGetSymbolAddress, with
- * that device current) and should come before any stream capture.
+ * that device current) and should come before any stream capture.  Under lazy module
+ * loading (CUDA_MODULE_LOADING=LAZY, the CUDA 12 default) the array takes device memory
+ * on a device only once the library's module is first used there; under eager loading
+ * every context that loads the library holds the 40 MiB from the start.
  * All calls on a device share the one array: calls that overlap in time (on different
  * streams, or from different host threads without ordering) race on it and corrupt each
  * other's results; calls ordered on one stream do not.  Nothing in the array needs to

@@ -23,6 +23,8 @@ struct AttnArgs {
   int tiles_per_batch;
   int bn;                   // keys per block of the launch
   int pf;                   // L2 look-ahead of the key loads in blocks (0: none)
+  float xthr;               // largest raw partial score magnitude a row's 16-bit score
+                            // exchange carries; a row with a larger one is sent exactly
   unsigned int* err;
 };
 

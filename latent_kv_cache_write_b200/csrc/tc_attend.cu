@@ -11,11 +11,13 @@
 //   - TMA-loads its columns of the 64 cached rows (one load serves as K and as V),
 //   - computes its partial score S_c = Q_c . K_c^T with tcgen05.mma (Q's latent half
 //     resident in TMEM as the A operand, the RoPE part from shared memory),
-//   - swaps partial scores (rounded to fp16) with its peer through distributed shared
-//     memory, so both CTAs hold the full scores of all 128 rows,
+//   - swaps partial scores with its peer through distributed shared memory, so both
+//     CTAs hold the full scores of all 128 rows: a row's partials go rounded to fp16
+//     while none exceeds a bound (a few tenths of a percent of a softmax weight at most),
+//     else as exact fp32 in two rounds,
 //   - runs the online softmax of all 128 rows itself (its own fp32 partial plus the
-//     peer's fp16-rounded one; the CTAs' row sums may differ in the last bits, and each
-//     normalises its own half of O with its own sum),
+//     peer's; the CTAs' row sums may differ in the last bits, and each normalises its own
+//     half of O with its own sum),
 //   - accumulates O_c += P . V_c (M=128, N=256) into its TMEM.
 //
 // Two softmax warpgroups take alternate key blocks, so the exchange of one block
@@ -106,7 +108,7 @@ struct Lay {
                                                 // after the scores)                      [NST]
   static constexpr int NBAR = B_KRE + NST;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr int SMEM = OFF_MISC + 48 + 1024;   // TMEM slot, abort flag, votes [2][4]
   static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
 };
 
@@ -180,6 +182,40 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
+// s[0..7] += the eight fp16 values packed in x (key 0 in the low half of x.x).
+__device__ __forceinline__ void add_f16x8(const uint4& x, float* s) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+    s[2 * e] += f.x;
+    s[2 * e + 1] += f.y;
+  }
+}
+
+// s[0..7] -= the eight fp16 values packed in x.
+__device__ __forceinline__ void sub_f16x8(const uint4& x, float* s) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+    s[2 * e] -= f.x;
+    s[2 * e + 1] -= f.y;
+  }
+}
+
+// This thread's row of a 64-column S buffer (fp32 partial scores) -> s.
+__device__ __forceinline__ void load_scores(uint32_t taddr, float (&s)[64]) {
+  uint32_t v[2][32];
+  tmem_ld32(taddr, v[0]);
+  tmem_ld32(taddr + 32, v[1]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int c = 0; c < 32; ++c) s[32 * h + c] = __uint_as_float(v[h][c]);
+}
+
 // Q latent half of row `grow` -> TMEM columns from `tq` (A operand of the score MMA),
 // bf16 pairs per column; each warpgroup loads half of the row.  All 16 vector loads are
 // issued before the first TMEM store, so their latencies overlap.
@@ -251,6 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bar[B_M + q], 128);
     }
     *abort = 0;
+    for (int q = 0; q < 8; ++q) reinterpret_cast<uint32_t*>(sm + LY::OFF_MISC + 16)[q] = 0u;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -448,6 +485,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     uint8_t* prow = sm + OFF_P + wg * XP_BYTES + t * (BN * 2);   // P row t
     const float c2 = a.scale_log2;
     bool ok = true;
+    uint32_t xc = 0;        // exchange rounds this warpgroup has taken part in (barrier phases)
+    uint32_t nd = 0;        // blocks this warpgroup has decided the exchange of
+    uint32_t* xvote = reinterpret_cast<uint32_t*>(sm + LY::OFF_MISC + 16);
 
     if (sw.valid()) {
       load_q(a, tmem + lane_base + Q_COL, sw.tg.grow0 + t, sw.tg.row0 + t < sw.tg.rows_b, rank,
@@ -480,8 +520,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int j = sw.jb + jl;              // block of the tile
         const int seq = sw.done_by(wg) + (jl >> 1);
         const uint32_t kph = seq & 1;
-        // arm this block's exchange: the peer's asynchronous stores complete XP_BYTES of
-        // transactions on it (they may land before or after this arrive)
+        // arm this block's first exchange round: the peer's asynchronous stores complete
+        // XP_BYTES of transactions on it (they may land before or after this arrive)
         if (t == 0) mbar_expect_tx(&bar[B_XF + wg], XP_BYTES);
         if (!__all_sync(FULL, mbar_wait(&bar[B_SF + wg], kph, abort, a.err, 0x201, (t << 16) | j))) {
           ok = false;
@@ -489,38 +529,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_after();
         float s[BN];
-        {
-          uint32_t v[BN / 32][32];
-#pragma unroll
-          for (int h = 0; h < BN / 32; ++h) tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32 * h, v[h]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < BN / 32; ++h)
-#pragma unroll
-            for (int c = 0; c < 32; ++c) s[32 * h + c] = __uint_as_float(v[h][c]);
-        }
+        load_scores(tmem + lane_base + S_COL + wg * BN, s);
         tc_fence_before();
         mbar_arrive(&bar[B_SE + wg]);
 
         // send this CTA's partial scores into the peer's buffer once the peer is done
-        // with it: it has read what was sent two blocks ago (and, with merged buffers,
-        // its PV has read the P held there)
-        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], kph ^ 1, abort, a.err, 0x202,
-                                                 (t << 16) | j))) {
+        // with it: it has read what was sent in this warpgroup's previous round (and,
+        // with merged buffers, its PV has read the P held there)
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], (xc & 1) ^ 1, abort, a.err,
+                                                 0x202, (t << 16) | j))) {
           ok = false;
           break;
         }
-        // the peer receives this partial rounded to fp16 (~2^-11 of a partial score)
-        uint32_t hs[BN / 2];
+        // The partials go rounded to fp16 (saturating: within 2^-11 of each partial).  A row
+        // with a partial beyond a.xthr in magnitude sets bit 0 of its last 16-byte chunk (the
+        // lowest mantissa bit of key 56), found while the first seven chunks travel; if any
+        // row of either CTA did, both CTAs' warpgroups exchange exact fp32 partials below.
+        bool need;
+        {
+          uint32_t hs[BN / 2];
 #pragma unroll
-        for (int c = 0; c < BN / 2; ++c) {
-          __half2 h2 = __floats2half2_rn(s[2 * c], s[2 * c + 1]);
-          hs[c] = *reinterpret_cast<uint32_t*>(&h2);
+          for (int c = 0; c < BN / 2; ++c) hs[c] = f16x2_satfinite(s[2 * c], s[2 * c + 1]);
+#pragma unroll
+          for (int q = 0; q < BN / 8 - 1; ++q)
+            st_async_v4(peer_x + q * (TM * 16), hs[4 * q], hs[4 * q + 1], hs[4 * q + 2],
+                        hs[4 * q + 3], peer_xf);
+          float hi[4], lo[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            hi[c] = fmax3(s[16 * c], s[16 * c + 1], s[16 * c + 2]);
+            lo[c] = fmin3(s[16 * c], s[16 * c + 1], s[16 * c + 2]);
+#pragma unroll
+            for (int e = 3; e < 15; e += 2) {
+              hi[c] = fmax3(hi[c], s[16 * c + e], s[16 * c + e + 1]);
+              lo[c] = fmin3(lo[c], s[16 * c + e], s[16 * c + e + 1]);
+            }
+            hi[c] = fmaxf(hi[c], s[16 * c + 15]);
+            lo[c] = fminf(lo[c], s[16 * c + 15]);
+          }
+          need = fmaxf(fmax3(hi[0], hi[1], fmaxf(hi[2], hi[3])),
+                       -fmin3(lo[0], lo[1], fminf(lo[2], lo[3]))) > a.xthr;
+          constexpr int QL = BN / 8 - 1;
+          st_async_v4(peer_x + QL * (TM * 16), (hs[4 * QL] & ~1u) | (need ? 1u : 0u),
+                      hs[4 * QL + 1], hs[4 * QL + 2], hs[4 * QL + 3], peer_xf);
         }
-#pragma unroll
-        for (int q = 0; q < BN / 8; ++q)
-          st_async_v4(peer_x + q * (TM * 16), hs[4 * q], hs[4 * q + 1], hs[4 * q + 2],
-                      hs[4 * q + 3], peer_xf);
 
         int64_t slot0, g0;
         int valid;
@@ -539,7 +591,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
 
         // full scores: add the peer's partial
-        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + wg], kph, abort, a.err, 0x203,
+        if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + wg], xc & 1, abort, a.err, 0x203,
                                                  (t << 16) | j))) {
           ok = false;
           break;
@@ -547,17 +599,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int q = 0; q < BN / 8; ++q) {
           const uint4 x = my_x[q * TM];
-          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-            s[8 * q + 2 * e] += f.x;
-            s[8 * q + 2 * e + 1] += f.y;
-          }
+          if (q == BN / 8 - 1) need = need || (x.x & 1u) != 0u;
+          add_f16x8(x, s + 8 * q);
         }
-        named_bar(1 + wg, TM);            // the whole buffer is read
-        if constexpr (!LY::MERGED) {
-          if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);   // hand it back
+        ++xc;
+        // The decision: a word per warpgroup and block (four in turn, each cleared two blocks
+        // before its next use) collects the rows' flags across the barrier that also
+        // marks the buffer as read.  Both CTAs see the same pairs of flags.
+        volatile uint32_t* vote = xvote + wg * 4;
+        if (need) atomicOr(const_cast<uint32_t*>(&vote[nd & 3]), 1u);
+        named_bar(1 + wg, TM);
+        const bool exact = vote[nd & 3] != 0u;
+        if (t == 0) vote[(nd + 2) & 3] = 0u;
+        ++nd;
+        if (exact) {
+          // Rounds two and three: undo the fp16 addend (s then holds this CTA's partial to
+          // within one float32 rounding) and swap exact fp32 partials, keys 0-31 then 32-63.
+#pragma unroll
+          for (int q = 0; q < BN / 8; ++q) sub_f16x8(my_x[q * TM], s + 8 * q);
+          named_bar(1 + wg, TM);                 // the buffer is read again before hand-back
+          if (t == 0) {
+            mbar_expect_tx(&bar[B_XF + wg], XP_BYTES);
+            mbar_arrive_cluster_relaxed(peer_xe);
+          }
+          for (int h = 0; ok && h < 2; ++h) {
+            if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XE + wg], (xc & 1) ^ 1, abort, a.err,
+                                                     0x207, (t << 16) | j))) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int q = 0; q < BN / 8; ++q)
+              st_async_v4(peer_x + q * (TM * 16), __float_as_uint(s[32 * h + 4 * q]),
+                          __float_as_uint(s[32 * h + 4 * q + 1]),
+                          __float_as_uint(s[32 * h + 4 * q + 2]),
+                          __float_as_uint(s[32 * h + 4 * q + 3]), peer_xf);
+            if (!__all_sync(FULL, mbar_wait_cluster(&bar[B_XF + wg], xc & 1, abort, a.err, 0x208,
+                                                     (t << 16) | j))) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int q = 0; q < BN / 8; ++q) {
+              const uint4 x = my_x[q * TM];
+              s[32 * h + 4 * q] += __uint_as_float(x.x);
+              s[32 * h + 4 * q + 1] += __uint_as_float(x.y);
+              s[32 * h + 4 * q + 2] += __uint_as_float(x.z);
+              s[32 * h + 4 * q + 3] += __uint_as_float(x.w);
+            }
+            ++xc;
+            named_bar(1 + wg, TM);
+            if (h == 0 && t == 0) mbar_expect_tx(&bar[B_XF + wg], XP_BYTES);   // round three
+            // with merged buffers the last round's buffer is handed back by the PV commit
+            if (!LY::MERGED || h == 0) {
+              if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);
+            }
+          }
+          if (!ok) break;
+        } else if constexpr (!LY::MERGED) {
+          if (t == 0) mbar_arrive_cluster_relaxed(peer_xe);   // hand the buffer back
         }
 
         // masked raw maximum (scores are scaled inside the exponent)
@@ -567,9 +667,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
-        float rmax = s[0];
+        float rm[4];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) rmax = fmaxf(rmax, s[c]);
+        for (int c = 0; c < 4; ++c) rm[c] = s[c];
+#pragma unroll
+        for (int c = 4; c < BN; c += 8) {
+          rm[0] = fmax3(rm[0], s[c], s[c + 1]);
+          rm[1] = fmax3(rm[1], s[c + 2], s[c + 3]);
+          rm[2] = fmax3(rm[2], s[c + 4], s[c + 5]);
+          rm[3] = fmax3(rm[3], s[c + 6], s[c + 7]);
+        }
+        const float rmax = fmaxf(fmax3(rm[0], rm[1], rm[2]), rm[3]);
         const float mb = rmax * c2;
 
         // running maximum after the previous block (published by the other warpgroup)
@@ -595,14 +703,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
         const float msub = m == -INFINITY ? 0.f : m;
         uint32_t pk[BN / 2];
-        float sum = 0.f;
+        float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < BN / 2; ++c) {
           const float p0 = ex2(fmaf(s[2 * c], c2, -msub));
           const float p1 = ex2(fmaf(s[2 * c + 1], c2, -msub));
-          sum += p0 + p1;
+          sums[c & 3] += p0 + p1;
           pk[c] = pack_bf16(p0, p1);
         }
+        const float sum = (sums[0] + sums[1]) + (sums[2] + sums[3]);
         l = l * ex2(m_last - msub) + sum;
         m_last = m;
         // O is rescaled (warp-collective TMEM access) after PV of the previous block.
@@ -718,8 +827,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     // with merged buffers the peer's last PV commit arrives on this CTA's barrier: let it
     // land before exit
     if constexpr (LY::MERGED) {
-      if (ok && !sw.valid() && sw.done_by(wg) > 0)
-        mbar_wait_cluster(&bar[B_XE + wg], (sw.done_by(wg) - 1) & 1, abort, a.err, 0x402, t);
+      if (ok && !sw.valid() && xc > 0)
+        mbar_wait_cluster(&bar[B_XE + wg], (xc - 1) & 1, abort, a.err, 0x402, t);
     }
   }
 
@@ -820,6 +929,16 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.g = g;
   a.n_q = n_q; a.q_first = q_first; a.k_first = k_first; a.n_keys = n_keys;
   a.scale_log2 = scale * 1.4426950408889634f;
+  {
+    // The 16-bit exchange rounds a partial score to within 2^-11 of itself.  Up to
+    // XCHG_LOG2 in the exponent's log2 units that error stays below 2^-8 of one such unit
+    // (a few tenths of a percent of a softmax weight, like the bf16 rounding of P); rows
+    // with larger partials get the exact exchange.  Capped well inside the fp16 range.
+    constexpr float XCHG_LOG2 = 8.f;
+    float thr = XCHG_LOG2 / a.scale_log2;
+    if (!(thr <= 32768.f)) thr = 32768.f;
+    a.xthr = thr;
+  }
   a.q_abs = (const bf16*)q_abs;
   a.o_lat = (bf16*)o_lat;
   a.lse = lse;
@@ -853,6 +972,15 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     }
   }
 
+  // Every group's schedule is built and checked before the first launch, so an error
+  // leaves nothing enqueued.
+  struct Plan {
+    Sched sc;
+    CombineList cl;
+    int G;
+  };
+  std::vector<Plan> plans;
+  bool any_partial = false;
   for (int b0 = 0; b0 < g.B; b0 += group) {
     const int t_lo = b0 * tiles_per_batch;
     const int t_hi = (b0 + group < g.B ? b0 + group : g.B) * tiles_per_batch;
@@ -947,22 +1075,25 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     }
     cl.piece0[cl.n] = nslot;
     if (nslot > 2 * ncl) return cudaErrorInvalidValue;    // at most two per cluster
-    if (nslot > 0) {
-      a.ws_o = (bf16*)workspace;
-      a.ws_lse = reinterpret_cast<float*>(a.ws_o + (size_t)2 * ncl * TM * g.Dc);
-    }
+    any_partial = any_partial || nslot > 0;
     if (G == 0) continue;
     for (int c = 0; c <= G; ++c) sc.cut_tile[c] += t_lo;
-
+    plans.push_back(Plan{sc, cl, G});
+  }
+  if (any_partial) {
+    a.ws_o = (bf16*)workspace;
+    a.ws_lse = reinterpret_cast<float*>(a.ws_o + (size_t)2 * ncl * TM * g.Dc);
+  }
+  for (const Plan& p : plans) {
     if (variant == 1)
-      attend_kernel<1><<<(unsigned)(2 * G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, sc);
+      attend_kernel<1><<<(unsigned)(2 * p.G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, p.sc);
     else
-      attend_kernel<0><<<(unsigned)(2 * G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, sc);
+      attend_kernel<0><<<(unsigned)(2 * p.G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, p.sc);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
-    if (cl.n > 0) {
-      e = launch_combine(a, cl, st);
+    if (p.cl.n > 0) {
+      e = launch_combine(a, p.cl, st);
       if (e != cudaSuccess) return e;
       count_launches(1);
     }

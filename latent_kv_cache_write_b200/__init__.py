@@ -31,14 +31,14 @@ import ctypes
 from typing import Optional
 
 from . import native
-from .native import MlaError, MlaShape, make_shape  # noqa: F401
+from .native import MLA_FIXED_SCRATCH_BYTES, MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
            "mla_attend_fixed_scratch", "mla_attend_materialised", "mla_cache_shift_frames",
            "mla_cache_quantise", "mla_cache_dequantise",
            "mla_attend_materialised_workspace_size", "mla_up_v", "mla_device_error",
            "mla_kernel_launches", "mla_device_error_info", "mla_check_wait_timeout", "make_shape",
-           "MlaShape", "MlaError"]
+           "MlaShape", "MlaError", "MLA_FIXED_SCRATCH_BYTES"]
 
 
 def _ptr(t) -> Optional[int]:

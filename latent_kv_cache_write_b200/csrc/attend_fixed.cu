@@ -1,7 +1,8 @@
 // Fixed device scratch for mla_attend_fixed_scratch: the split-key partials of the
 // attention kernel in a static device array instead of a caller workspace.  It lives in
-// its own translation unit, so the array is set up on a device only when this entry
-// point is first used there.
+// its own translation unit.  Under lazy module loading (the CUDA 12 default) the array
+// takes device memory on a device only once the module is first used there; under eager
+// loading (CUDA_MODULE_LOADING=EAGER) every context that loads the library holds it.
 #include "launch.h"
 
 #include <mutex>

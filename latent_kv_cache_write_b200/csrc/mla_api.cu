@@ -3,6 +3,7 @@
 #include <stdio.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "launch.h"
 
@@ -18,15 +19,15 @@ void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order
 
 unsigned int* device_error_word() {
   // One lookup per device: the symbol's address differs between devices.
+  static std::mutex mu;
   static unsigned int* addr[64] = {};
-  static std::atomic<int> done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!done[dev].load(std::memory_order_acquire)) {
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
     addr[dev] = static_cast<unsigned int*>(p);
-    done[dev].store(1, std::memory_order_release);
   }
   return addr[dev];
 }
@@ -85,6 +86,38 @@ mla_status check_quant(const mla_shape* shape, Geo* g, int64_t first_tok, int64_
       !aligned16(sr))
     return MLA_ERR_ALIGN;
   return MLA_OK;
+}
+
+// the checks of mla_attend and mla_attend_fixed_scratch, all but the workspace's
+mla_status check_attend(const mla_shape* shape, Geo* g, const void* q_abs, int64_t n_q,
+                        int64_t q_first_tok, const void* cache, int64_t k_first_tok,
+                        int64_t n_keys, float softmax_scale, const void* o_lat,
+                        const float* lse) {
+  mla_status st = check_shape(shape, g);
+  if (st != MLA_OK) return st;
+  if (n_q < 0 || !q_abs || !cache || !o_lat) return MLA_ERR_ARG;
+  if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return MLA_ERR_ARG;
+  if (n_keys < 1 || n_keys > g->S || k_first_tok < 0 || q_first_tok < k_first_tok ||
+      q_first_tok + n_q > k_first_tok + n_keys)
+    return MLA_ERR_RANGE;
+  if (n_q > 65535 || (int64_t)g->B * n_q * g->H > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(o_lat) || (lse && !aligned16(lse)))
+    return MLA_ERR_ALIGN;
+  return MLA_OK;
+}
+
+// the launches of a checked attention call (n_q > 0)
+mla_status run_attend(const mla_shape* shape, const Geo& g, const void* q_abs, int64_t n_q,
+                      int64_t q_first_tok, const void* cache, int64_t k_first_tok,
+                      int64_t n_keys, float softmax_scale, void* o_lat, float* lse,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  const bool bf = shape->dtype == MLA_BF16;
+  if (bf && tc_attend_supported(g))
+    return cuda_status(tc_attend(g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                                 softmax_scale, o_lat, lse, workspace, workspace_bytes,
+                                 device_error_word(), (cudaStream_t)stream));
+  return cuda_status(simt_attend(g, bf, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                                 softmax_scale, o_lat, lse, (cudaStream_t)stream));
 }
 
 }  // namespace
@@ -164,16 +197,9 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
                       int64_t n_keys, float softmax_scale, void* o_lat, float* lse,
                       void* workspace, size_t workspace_bytes, void* stream) {
   Geo g;
-  mla_status st = check_shape(shape, &g);
+  mla_status st = check_attend(shape, &g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                               softmax_scale, o_lat, lse);
   if (st != MLA_OK) return st;
-  if (n_q < 0 || !q_abs || !cache || !o_lat) return MLA_ERR_ARG;
-  if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return MLA_ERR_ARG;
-  if (n_keys < 1 || n_keys > g.S || k_first_tok < 0 || q_first_tok < k_first_tok ||
-      q_first_tok + n_q > k_first_tok + n_keys)
-    return MLA_ERR_RANGE;
-  if (n_q > 65535 || (int64_t)g.B * n_q * g.H > INT32_MAX) return MLA_ERR_UNSUPPORTED;
-  if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(o_lat) || (lse && !aligned16(lse)))
-    return MLA_ERR_ALIGN;
   // no workspace at all is allowed (the schedule then keeps tiles whole); a workspace
   // that is given must be large enough
   const size_t need = mla_attend_workspace_size(shape, n_q, n_keys);
@@ -181,13 +207,8 @@ mla_status mla_attend(const mla_shape* shape, const void* q_abs, int64_t n_q,
     return MLA_ERR_ARG;
   if (workspace && !aligned16(workspace)) return MLA_ERR_ALIGN;
   if (n_q == 0) return MLA_OK;
-  const bool bf = shape->dtype == MLA_BF16;
-  if (bf && tc_attend_supported(g))
-    return cuda_status(tc_attend(g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
-                                 softmax_scale, o_lat, lse, workspace, workspace_bytes,
-                                 device_error_word(), (cudaStream_t)stream));
-  return cuda_status(simt_attend(g, bf, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
-                                 softmax_scale, o_lat, lse, (cudaStream_t)stream));
+  return run_attend(shape, g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                    softmax_scale, o_lat, lse, workspace, workspace_bytes, stream);
 }
 
 mla_status mla_attend_fixed_scratch(const mla_shape* shape, const void* q_abs, int64_t n_q,
@@ -195,8 +216,10 @@ mla_status mla_attend_fixed_scratch(const mla_shape* shape, const void* q_abs, i
                                     int64_t k_first_tok, int64_t n_keys, float softmax_scale,
                                     void* o_lat, float* lse, void* stream) {
   Geo g;
-  mla_status st = check_shape(shape, &g);
+  mla_status st = check_attend(shape, &g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                               softmax_scale, o_lat, lse);
   if (st != MLA_OK) return st;
+  if (n_q == 0) return MLA_OK;
   // the static array replaces the caller's workspace; a shape and device that would
   // need more is refused rather than run with a smaller schedule
   const size_t need = mla_attend_workspace_size(shape, n_q, n_keys);
@@ -207,8 +230,8 @@ mla_status mla_attend_fixed_scratch(const mla_shape* shape, const void* q_abs, i
     if (fixed_scratch(&scratch) != cudaSuccess) return MLA_ERR_CUDA;
     bytes = MLA_FIXED_SCRATCH_BYTES;
   }
-  return mla_attend(shape, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys, softmax_scale,
-                    o_lat, lse, scratch, bytes, stream);
+  return run_attend(shape, g, q_abs, n_q, q_first_tok, cache, k_first_tok, n_keys,
+                    softmax_scale, o_lat, lse, scratch, bytes, stream);
 }
 
 mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, const void* w_uv,

@@ -16,6 +16,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so"
 MLA_OK, MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_ALIGN, MLA_ERR_RANGE, MLA_ERR_CUDA, \
     MLA_ERR_TIMEOUT = range(7)
 MLA_F32, MLA_BF16 = 0, 1
+MLA_FIXED_SCRATCH_BYTES = 40 * 1024 * 1024     # the header's static split-key scratch
 
 # Every symbol the header declares, with (restype, argtypes).
 _vp, _i32, _i64, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,

@@ -42,5 +42,15 @@ int main(void) {
   printf("empty_dequant %s\n",
          mla_status_string(mla_cache_dequantise(&s, fake, fake, fs, fs, 2, 4, 0, 0, fake,
                                                 NULL)));
+  /* the no-workspace attention: checked like mla_attend, an empty call succeeds */
+  printf("fixed_range %s\n",
+         mla_status_string(mla_attend_fixed_scratch(&s, fake, 1560, 3 * 1560 + 1, fake, 0,
+                                                    6240, 0.07f, fake, NULL, NULL)));
+  printf("fixed_align %s\n",
+         mla_status_string(mla_attend_fixed_scratch(&s, fake + 8, 1560, 3 * 1560, fake, 0,
+                                                    6240, 0.07f, fake, NULL, NULL)));
+  printf("fixed_empty %s\n",
+         mla_status_string(mla_attend_fixed_scratch(&s, fake, 0, 0, fake, 0, 6240, 0.07f, fake,
+                                                    NULL, NULL)));
   return 0;
 }

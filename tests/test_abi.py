@@ -225,3 +225,35 @@ def test_row_counts_beyond_32_bit_coordinates(L):
     big = _shape(batch=1000, n_heads=65, ring_slots=50000)    # 1000 x 40000 x 65 rows
     assert _attend(L, big, n_q=40000, q_first=0, n_keys=50000) == U
     assert _mat(L, big, n_q=40000, q_first=0, n_keys=50000, ws_bytes=1 << 62) == U
+
+
+def _fixed(L, s, q=FAKE, n_q=1560, q_first=3 * 1560, cache=FAKE, k_first=0, n_keys=6240,
+           scale=0.07, o=FAKE, lse=None):
+    return L.mla_attend_fixed_scratch(ctypes.byref(s), q, n_q, q_first, cache, k_first, n_keys,
+                                      scale, o, lse, None)
+
+
+def test_fixed_scratch_validation(L):
+    """The no-workspace entry point answers bad arguments exactly as mla_attend does,
+    before it looks up its static array or launches anything."""
+    s = _shape()
+    assert native.MLA_FIXED_SCRATCH_BYTES == 40 * 1024 * 1024
+    assert "#define MLA_FIXED_SCRATCH_BYTES (40u * 1024u * 1024u)" in open(HEADER).read()
+    R, A = native.MLA_ERR_RANGE, native.MLA_ERR_ARG
+    assert _fixed(L, _shape(batch=0)) == A
+    assert _fixed(L, _shape(dtype=7)) == native.MLA_ERR_UNSUPPORTED
+    assert L.mla_attend_fixed_scratch(None, FAKE, 1, 0, FAKE, 0, 1, 1.0, FAKE, None, None) == A
+    assert _fixed(L, s, n_keys=6241) == R
+    assert _fixed(L, s, n_keys=0) == R
+    assert _fixed(L, s, k_first=-1) == R
+    assert _fixed(L, s, q_first=3 * 1560 + 1) == R
+    assert _fixed(L, s, q=None) == A
+    assert _fixed(L, s, cache=None) == A
+    assert _fixed(L, s, o=None) == A
+    assert _fixed(L, s, scale=float("nan")) == A
+    assert _fixed(L, s, n_q=-1) == A
+    assert _fixed(L, s, q=ODD) == native.MLA_ERR_ALIGN
+    assert _fixed(L, s, lse=ODD) == native.MLA_ERR_ALIGN
+    assert _fixed(L, s, n_q=0) == native.MLA_OK               # empty: nothing to do
+    big = _shape(batch=1000, n_heads=65, ring_slots=50000)
+    assert _fixed(L, big, n_q=40000, q_first=0, n_keys=50000) == native.MLA_ERR_UNSUPPORTED

@@ -23,7 +23,7 @@ def test_plain_c_host(tmp_path):
                    check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True,
                          timeout=120).stdout.split("\n")
-    assert out[:8] == [
+    assert out[:11] == [
         "status MLA_ERR_RANGE",
         f"materialised_ws {2 * 6240 * 32 * 128 * 2}",
         "attend_range MLA_ERR_RANGE",
@@ -32,4 +32,7 @@ def test_plain_c_host(tmp_path):
         "empty_shift MLA_OK",
         "quant_bits MLA_ERR_ARG",
         "empty_dequant MLA_OK",
+        "fixed_range MLA_ERR_RANGE",
+        "fixed_align MLA_ERR_ALIGN",
+        "fixed_empty MLA_OK",
     ]

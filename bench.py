@@ -463,6 +463,33 @@ def decode_leg(torch, mla, steps, warmup, flush, wl=C.DECODE):
             "tflops": step_flops(wl)["attend"] / (t * 1e-3) / 1e12}
 
 
+def workload_leg(torch, mla, name, steps, warmup, flush, peaks, device):
+    """The whole step (cache write of the chunk, absorption, attention, up-projection) of
+    another workload, timed like the main step with the L2 flushed before each one; the
+    attention's rate against the measured bf16 peak, with the clocks seen meanwhile."""
+    wl = C.BY_NAME[name]
+    step = Step(wl, seed=0, torch=torch, mla=mla)
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    with ClockSampler(device) as clocks:
+        ms, parts = time_steps(torch, lambda ev: step.run(ev=ev), steps, flush, n_marks=5)
+    torch.cuda.synchronize()
+    kms = {k: statistics.mean(v) for k, v in zip(Step.STAGES, parts)}
+    fl = step_flops(wl)
+    att = fl["attend"] / (kms["attend"] * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    out = {"workload": wl.name, "config": step_config(wl, 1), "steps": steps,
+           "ms_per_step": statistics.mean(ms),
+           "tflops_per_step": sum(fl.values()) / (statistics.mean(ms) * 1e-3) / 1e12,
+           "attend": {"ms": kms["attend"], "flops": fl["attend"], "tflops": att, "peak": peak,
+                      "frac": att / peak, "p10_p50_p90": percentiles(dict(zip(Step.STAGES, parts))["attend"])},
+           "kernels_ms": kms, "clocks": clocks.summary()}
+    del step
+    torch.cuda.empty_cache()
+    return out
+
+
 _CPU_STATE = {}
 
 
@@ -527,11 +554,10 @@ def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
             "seconds": dt}
 
 
-# DRAM bytes (read + write) of one chunk mla_attend call, from the ncu captures summarised in
-# profiles/attend_kernel_video_chunk.md (the attention kernel) and
-# profiles/combine_kernel_video_chunk.md (the split-key merge).  Counters describe the kernel
-# sources they were taken on (the two kernels and the headers they compile in): the value is
-# reported only while those sources are unchanged.
+# DRAM bytes (read + write) of one chunk mla_attend call, from one ncu capture of the
+# attention kernel and one of its split-key merge.  Counters describe the kernel sources they
+# were taken on (the two kernels and the headers they compile in): the value is reported
+# only while those sources are unchanged.
 ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
                   "bytes": (72_785_152 + 18_896_384) + (19_032_576 + 0),
                   "sources": {
@@ -643,6 +669,11 @@ def run_ours(args):
     if dec:
         dec["peak_gbs"] = float(peaks["hbm_gbs"])
         dec["frac"] = dec["value"] / dec["peak_gbs"]
+    # the long-window and wide-positional-key steps, in the same run
+    others = {n: workload_leg(torch, mla, n, max(3, min(args.steps, 10)), args.warmup, flush,
+                              peaks, local)
+              for n in ("long_window_bf16", "wide_key_bf16") if n != wl.name} \
+        if rank == 0 else None
     if rank == 0:
         line = {
             "metric": "absorbed MLA attention TFLOP/s (chunk) and latent-cache GB/s (decode) "
@@ -675,6 +706,7 @@ def run_ours(args):
             "materialised": mat,
             "k_rope_shift": shift,
             "quant_ring": quant,
+            "workloads": others,
             "clocks": clocks.summary(),
             "kernels_ms": kernels_ms,
         }

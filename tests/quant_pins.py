@@ -16,6 +16,7 @@ import numpy as np
 
 import oracle.latent_quant as QZ
 import oracle.mla_oracle as O
+from synth import configs as C
 from synth import generate as G
 from tests import oracle_pins as P
 
@@ -208,6 +209,56 @@ def pin_quant_bytes():
         wl.d_latent, wl.d_rope, 2, 4)
 
 
+def _video_chunk_window_rows() -> np.ndarray:
+    """The 6240 rows of the video-chunk window (frames 0-3 through the oracle's cache
+    write), rounded to bf16 as the ring holds them."""
+    wl = C.VIDEO_CHUNK
+    w = G.weights(wl, 0)
+    F = wl.tokens_per_frame
+    rows = [O.cache_rows(G.hidden_frame(wl, 0, f).values, w["w_dkv"].values,
+                         w["w_kr"].values, f * F, wl)[0] for f in range(4)]
+    return G.to_storage(np.concatenate(rows), "bf16").values
+
+
+DECISION_DIFFS = {}        # (bits, path) -> codes the float32 decision changes, on the window
+
+
+def pin_quant_float32_decision():
+    """x / s evaluated in float32 (as a float32 kernel does) against the exact decision:
+    the scale is the same, codes differ by at most one, and only where x / s lies within
+    float32 rounding of a half-integer (the division's result within 2^-24 of itself, the
+    bf16 x exact in float32).  Counted on every element of the video-chunk window at 2, 4
+    and 8 bits (DECISION_DIFFS); then on constructed near-ties where the two do differ."""
+    rows = _video_chunk_window_rows()
+    d_c = C.VIDEO_CHUNK.d_latent
+    for bits in (2, 4, 8):
+        for path, x in (("content", rows[:, :d_c]), ("rope", rows[:, d_c:])):
+            c64, s64 = QZ.quantise_rows(x, bits)
+            c32, s32 = QZ.quantise_rows(x, bits, decide=np.float32)
+            assert np.array_equal(s64, s32)
+            diff = c64.astype(np.int64) - c32.astype(np.int64)
+            assert np.abs(diff).max() <= 1, (bits, path)
+            DECISION_DIFFS[(bits, path)] = int(np.count_nonzero(diff))
+            for r, i in zip(*np.nonzero(diff)):
+                ratio = Fraction(float(x[r, i])) / Fraction(float(s64[r]))
+                off = abs(ratio - math.floor(ratio) - Fraction(1, 2))
+                assert off <= abs(ratio) * Fraction(1, 2 ** 22), (bits, path, r, i)
+    # near-ties: x just above (k + 1/2) s, where the float32 quotient rounds to the tie
+    rng = np.random.default_rng(5)
+    found = 0
+    for _ in range(2000):
+        s = float(np.float32(rng.uniform(0.01, 10.0)))
+        x = 2.5 * s * (1.0 + 2.0 ** -28)          # exact quotient a hair above 2.5
+        row = np.array([[7.0 * s, x]])            # max|x| / 7 = s exactly, so the scale is s
+        c64, sc = QZ.quantise_rows(row, 4)
+        c32, _ = QZ.quantise_rows(row, 4, decide=np.float32)
+        assert float(sc[0]) == s and c64[0, 1] == 3
+        if c32[0, 1] != c64[0, 1]:
+            assert c32[0, 1] == 2                 # the tie, to even: one code apart
+            found += 1
+    assert found > 0
+
+
 ALL_QUANT_PINS = [pin_quant_brute_force, pin_quant_error_bound, pin_quant_grid_exact,
                   pin_pack_layout, pin_quant_paths_separate, pin_quant_ring_write,
-                  pin_quant_attention_converges, pin_quant_bytes]
+                  pin_quant_attention_converges, pin_quant_bytes, pin_quant_float32_decision]

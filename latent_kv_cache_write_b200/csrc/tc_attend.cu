@@ -182,17 +182,6 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
-// s[0..7] += the eight fp16 values packed in x (key 0 in the low half of x.x).
-__device__ __forceinline__ void add_f16x8(const uint4& x, float* s) {
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-    s[2 * e] += f.x;
-    s[2 * e + 1] += f.y;
-  }
-}
-
 // s[0..7] -= the eight fp16 values packed in x.
 __device__ __forceinline__ void sub_f16x8(const uint4& x, float* s) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -600,7 +589,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int q = 0; q < BN / 8; ++q) {
           const uint4 x = my_x[q * TM];
           if (q == BN / 8 - 1) need = need || (x.x & 1u) != 0u;
-          add_f16x8(x, s + 8 * q);
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            s[8 * q + 2 * e] = add_f32_f16(s[8 * q + 2 * e], w[e] & 0xFFFFu);
+            s[8 * q + 2 * e + 1] = add_f32_f16(s[8 * q + 2 * e + 1], w[e] >> 16);
+          }
         }
         ++xc;
         // The decision: a word per warpgroup and block (four in turn, each cleared two blocks
@@ -667,17 +661,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
-        float rm[4];
+        float rm[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) rm[c] = s[c];
+        for (int c = 0; c < 8; ++c) rm[c] = s[c];
 #pragma unroll
-        for (int c = 4; c < BN; c += 8) {
-          rm[0] = fmax3(rm[0], s[c], s[c + 1]);
-          rm[1] = fmax3(rm[1], s[c + 2], s[c + 3]);
-          rm[2] = fmax3(rm[2], s[c + 4], s[c + 5]);
-          rm[3] = fmax3(rm[3], s[c + 6], s[c + 7]);
-        }
-        const float rmax = fmaxf(fmax3(rm[0], rm[1], rm[2]), rm[3]);
+        for (int c = 8; c < BN; ++c) rm[c & 7] = fmaxf(rm[c & 7], s[c]);
+        const float rmax = fmaxf(fmaxf(fmaxf(rm[0], rm[1]), fmaxf(rm[2], rm[3])),
+                                 fmaxf(fmaxf(rm[4], rm[5]), fmaxf(rm[6], rm[7])));
         const float mb = rmax * c2;
 
         // running maximum after the previous block (published by the other warpgroup)

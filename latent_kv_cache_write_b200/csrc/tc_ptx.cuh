@@ -389,7 +389,14 @@ __device__ __forceinline__ uint32_t f16x2_satfinite(float lo, float hi) {
   return d;
 }
 
-// max(a, b, c) and min(a, b, c) in one instruction each.
+// c + h with h an fp16 value (its bits), the sum rounded to float32: one instruction.
+__device__ __forceinline__ float add_f32_f16(float c, uint32_t h) {
+  float d;
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"((uint16_t)h), "f"(c));
+  return d;
+}
+
+// max(a, b, c) and min(a, b, c).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

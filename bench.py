@@ -490,6 +490,66 @@ def workload_leg(torch, mla, name, steps, warmup, flush, peaks, device):
     return out
 
 
+def quant_attend_leg(torch, mla, steps, warmup, flush, peaks, chunk_step=None):
+    """Attention with the dequantisation fused in (mla_attend_quantised): the decode
+    workload over its ring quantised to INT4 / INT4 and INT2 / INT4, and the video chunk
+    over an INT4 ring; bytes are those the call reads and writes (packed ring, q_abs, o_lat)."""
+    out = {}
+    wl = C.DECODE
+    shape = mla.make_shape(wl)
+    dev = "cuda"
+    up = lambda t: torch.from_numpy(t.storage.view(np.int16)).to(dev).view(torch.bfloat16)
+    cache = up(G.direct_cache(wl, 0))
+    q = G.queries(wl, 0)
+    w = G.weights(wl, 0)
+    q_abs = torch.empty((wl.batch, 1, wl.n_heads, wl.row_width), dtype=torch.bfloat16, device=dev)
+    mla.mla_absorb_q(shape, up(q["q_nope"]), up(q["q_rope"]), 1, wl.q_first_tok, up(w["w_uk"]),
+                     q_abs)
+
+    def run(shape, wl, q_abs, cache, T, cb, rb):
+        B, S = wl.batch, wl.ring_slots
+        qc = torch.empty((B, S, wl.d_latent * cb // 8), dtype=torch.uint8, device=dev)
+        qr = torch.empty((B, S, wl.d_rope * rb // 8), dtype=torch.uint8, device=dev)
+        sc = torch.empty((B, S), dtype=torch.float32, device=dev)
+        sr = torch.empty_like(sc)
+        mla.mla_cache_quantise(shape, cache, wl.k_first_tok, wl.n_keys, cb, rb, qc, qr, sc, sr)
+        o = torch.empty((B, T, wl.n_heads, wl.d_latent), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, T, wl.n_heads), dtype=torch.float32, device=dev)
+        nws = mla.mla_attend_workspace_size(shape, T, wl.n_keys)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+
+        def call(_a=None):
+            mla.mla_attend_quantised(shape, q_abs, T, wl.q_first_tok, qc, qr, sc, sr, cb, rb,
+                                     wl.k_first_tok, wl.n_keys, wl.softmax_scale, o, lse, ws,
+                                     nws)
+
+        for _ in range(warmup):
+            call()
+        ms, _ = time_steps(torch, call, steps, flush)
+        t = statistics.mean(ms)
+        tok = quant_token_bytes(wl, cb, rb)
+        moved = wl.batch * wl.n_keys * tok + q_abs.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+        return t, tok, moved
+
+    for cb, rb in ((4, 4), (2, 4)):
+        t, tok, moved = run(shape, wl, q_abs, cache, 1, cb, rb)
+        out[f"decode_c{cb}r{rb}"] = {
+            "workload": wl.name, "ms": t, "bytes": moved, "value": moved / (t * 1e-3) / 1e9,
+            "unit": "GB/s", "frac_hbm": moved / (t * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+            "bytes_per_token": tok, "capacity_vs_bf16": wl.row_width * 2 / tok,
+            "tflops": step_flops(wl)["attend"] / (t * 1e-3) / 1e12}
+    if chunk_step is not None:
+        st = chunk_step
+        t, tok, moved = run(st.shape, st.wl, st.q_abs, st.cache, st.wl.n_queries, 4, 4)
+        fl = step_flops(st.wl)["attend"]
+        out["video_chunk_c4r4"] = {"workload": st.wl.name, "ms": t, "tflops": fl / (t * 1e-3) / 1e12,
+                                   "frac": fl / (t * 1e-3) / 1e12 / float(peaks["bf16_tflops"]),
+                                   "bytes_per_token": tok}
+    out["note"] = ("mla_attend_quantised: two warps per CTA dequantise each block's packed rows "
+                   "into the K/V stage; decode reads the packed ring once")
+    return out
+
+
 _CPU_STATE = {}
 
 
@@ -669,6 +729,8 @@ def run_ours(args):
     if dec:
         dec["peak_gbs"] = float(peaks["hbm_gbs"])
         dec["frac"] = dec["value"] / dec["peak_gbs"]
+    qatt = quant_attend_leg(torch, mla, max(3, args.steps), args.warmup, flush, peaks, step) \
+        if rank == 0 else None
     # the long-window and wide-positional-key steps, in the same run
     others = {n: workload_leg(torch, mla, n, max(3, min(args.steps, 10)), args.warmup, flush,
                               peaks, local)
@@ -706,6 +768,7 @@ def run_ours(args):
             "materialised": mat,
             "k_rope_shift": shift,
             "quant_ring": quant,
+            "quant_attend": qatt,
             "workloads": others,
             "clocks": clocks.summary(),
             "kernels_ms": kernels_ms,

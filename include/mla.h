@@ -284,6 +284,38 @@ mla_status mla_cache_dequantise(const mla_shape* shape, const void* q_content,
                                 int64_t first_tok, int64_t n_tok, void* cache, void* stream);
 
 /*
+ * mla_attend_quantised — steps 3 and 4 over the low-bit ring, with the dequantisation inside
+ * the attention kernel (QuantMLA abstract on the "Multi-Head Latent Attention" topic page:
+ * the attention unpacks and dequantises the INT4 / INT2 content codes and the INT4 RoPE
+ * codes itself; the scores, softmax and output are those of mla_attend).
+ *
+ * The result is that of mla_attend over the ring whose rows are the dequantised values
+ *   cache[b][r][i] = code_i * scale[b][r]      (both paths, as mla_cache_dequantise defines
+ *                                              them),
+ * up to rounding: inside the kernel a row's scale is rounded to bf16 and each product
+ * code * scale to bf16 (the tensor cores' operand type), so an element can differ from the
+ * float32 product rounded once by a unit in the last bf16 place.
+ *
+ *   q_abs      [B, n_q, n_h, d_latent + d_rope]            read
+ *   q_content  [B, S, d_latent * content_bits / 8] bytes    read (mla_cache_quantise's layout)
+ *   q_rope     [B, S, d_rope * rope_bits / 8] bytes         read
+ *   scale_c, scale_r [B, S] float32                          read
+ *   o_lat, lse, workspace: as in mla_attend (the same workspace size)
+ * Supported: bfloat16, d_latent = 512, d_rope = 64, content_bits 4 or 2, rope_bits 4 (the
+ * two configurations the QuantMLA abstract names).
+ * Errors: those of mla_attend (the packed content codes stand where the cache does);
+ * MLA_ERR_ARG for a NULL q_rope or scale, or a bit width other than 2, 4, 8;
+ * MLA_ERR_UNSUPPORTED for other shapes, bit widths or float32; MLA_ERR_ALIGN for a pointer
+ * not 16-byte aligned.
+ */
+mla_status mla_attend_quantised(const mla_shape* shape, const void* q_abs, int64_t n_q,
+                                int64_t q_first_tok, const void* q_content, const void* q_rope,
+                                const float* scale_c, const float* scale_r,
+                                int32_t content_bits, int32_t rope_bits, int64_t k_first_tok,
+                                int64_t n_keys, float softmax_scale, void* o_lat, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * mla_attend_materialised_workspace_size — bytes of device workspace mla_attend_materialised
  * needs: the per-head keys and then the per-head values of every ring slot, bf16,
  * 2 * B * S * n_h * d_nope * 2 bytes.  0 for shapes the call does not support.

@@ -34,7 +34,8 @@ from . import native
 from .native import MLA_FIXED_SCRATCH_BYTES, MlaError, MlaShape, make_shape  # noqa: F401
 
 __all__ = ["mla_cache_write", "mla_absorb_q", "mla_attend", "mla_attend_workspace_size",
-           "mla_attend_fixed_scratch", "mla_attend_materialised", "mla_cache_shift_frames",
+           "mla_attend_fixed_scratch", "mla_attend_materialised", "mla_attend_quantised",
+           "mla_cache_shift_frames",
            "mla_cache_quantise", "mla_cache_dequantise",
            "mla_attend_materialised_workspace_size", "mla_up_v", "mla_device_error",
            "mla_kernel_launches", "mla_device_error_info", "mla_check_wait_timeout", "make_shape",
@@ -116,6 +117,20 @@ def mla_cache_dequantise(shape: MlaShape, q_content, q_rope, scale_c, scale_r,
     native.check("mla_cache_dequantise", native.lib().mla_cache_dequantise(
         ctypes.byref(shape), _ptr(q_content), _ptr(q_rope), _ptr(scale_c), _ptr(scale_r),
         content_bits, rope_bits, first_tok, n_tok, _ptr(cache), _stream(stream)))
+
+
+def mla_attend_quantised(shape: MlaShape, q_abs, n_q: int, q_first_tok: int, q_content, q_rope,
+                         scale_c, scale_r, content_bits: int, rope_bits: int, k_first_tok: int,
+                         n_keys: int, softmax_scale: float, o_lat, lse=None, workspace=None,
+                         workspace_bytes: Optional[int] = None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else (
+            workspace.numel() * workspace.element_size())
+    native.check("mla_attend_quantised", native.lib().mla_attend_quantised(
+        ctypes.byref(shape), _ptr(q_abs), n_q, q_first_tok, _ptr(q_content), _ptr(q_rope),
+        _ptr(scale_c), _ptr(scale_r), content_bits, rope_bits, k_first_tok, n_keys,
+        softmax_scale, _ptr(o_lat), _ptr(lse), _ptr(workspace), workspace_bytes,
+        _stream(stream)))
 
 
 def mla_attend_materialised_workspace_size(shape: MlaShape) -> int:

@@ -25,6 +25,12 @@ struct AttnArgs {
   int pf;                   // L2 look-ahead of the key loads in blocks (0: none)
   float xthr;               // largest raw partial score magnitude a row's 16-bit score
                             // exchange carries; a row with a larger one is sent exactly
+  // the low-bit ring (packed variant only): codes of both paths, per-row float32 scales
+  const uint8_t* pk_c;      // [B][S][d_c * cbits / 8]
+  const uint8_t* pk_r;      // [B][S][d_R * rbits / 8]
+  const float* sc_c;        // [B][S]
+  const float* sc_r;        // [B][S]
+  int cbits, rbits;
   unsigned int* err;
 };
 

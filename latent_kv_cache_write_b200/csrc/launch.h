@@ -73,6 +73,24 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
                       void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
                       unsigned int* err, cudaStream_t st);
 
+// The low-bit ring the attention reads instead of a bf16 cache (packed codes of both paths
+// and their per-row float32 scales, as mla_cache_quantise writes them).
+struct PackedRing {
+  const void* codes_c;
+  const void* codes_r;
+  const float* scale_c;
+  const float* scale_r;
+  int cbits, rbits;
+};
+// Content codes of 4 or 2 bits and RoPE codes of 4 bits, d_c = 512, d_R = 64.
+bool tc_attend_packed_supported(const Geo& g, int cbits, int rbits);
+// tc_attend over either ring: `cache` when pk is null, else the packed ring *pk.
+cudaError_t tc_attend_ring(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
+                           const void* cache, const PackedRing* pk, int64_t k_first,
+                           int64_t n_keys, float scale, void* o_lat, float* lse,
+                           void* workspace, size_t workspace_bytes, unsigned int* err,
+                           cudaStream_t st);
+
 // Address of the static split-key scratch (MLA_FIXED_SCRATCH_BYTES) on the current device.
 cudaError_t fixed_scratch(void** ptr);
 

@@ -234,6 +234,34 @@ mla_status mla_attend_fixed_scratch(const mla_shape* shape, const void* q_abs, i
                     softmax_scale, o_lat, lse, scratch, bytes, stream);
 }
 
+mla_status mla_attend_quantised(const mla_shape* shape, const void* q_abs, int64_t n_q,
+                                int64_t q_first_tok, const void* q_content, const void* q_rope,
+                                const float* scale_c, const float* scale_r,
+                                int32_t content_bits, int32_t rope_bits, int64_t k_first_tok,
+                                int64_t n_keys, float softmax_scale, void* o_lat, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  Geo g;
+  // the packed ring stands where mla_attend takes the bf16 cache
+  mla_status st = check_attend(shape, &g, q_abs, n_q, q_first_tok, q_content, k_first_tok,
+                               n_keys, softmax_scale, o_lat, lse);
+  if (st != MLA_OK) return st;
+  if (!q_rope || !scale_c || !scale_r || !quant_bits_ok(content_bits) ||
+      !quant_bits_ok(rope_bits))
+    return MLA_ERR_ARG;
+  if (shape->dtype != MLA_BF16 || !tc_attend_packed_supported(g, content_bits, rope_bits))
+    return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_rope) || !aligned16(scale_c) || !aligned16(scale_r)) return MLA_ERR_ALIGN;
+  const size_t need = mla_attend_workspace_size(shape, n_q, n_keys);
+  if ((workspace || workspace_bytes > 0) && (!workspace || workspace_bytes < need))
+    return MLA_ERR_ARG;
+  if (workspace && !aligned16(workspace)) return MLA_ERR_ALIGN;
+  if (n_q == 0) return MLA_OK;
+  const PackedRing pk{q_content, q_rope, scale_c, scale_r, content_bits, rope_bits};
+  return cuda_status(tc_attend_ring(g, q_abs, n_q, q_first_tok, nullptr, &pk, k_first_tok,
+                                    n_keys, softmax_scale, o_lat, lse, workspace,
+                                    workspace_bytes, device_error_word(), (cudaStream_t)stream));
+}
+
 mla_status mla_up_v(const mla_shape* shape, const void* o_lat, int64_t n_q, const void* w_uv,
                     void* out, void* stream) {
   Geo g;

@@ -54,15 +54,17 @@ namespace {
 using namespace tc;
 using namespace attn;
 
-constexpr int NTHREADS = 352;
-
-// Two variants of one kernel, chosen per call by the host; both take 64-key blocks.
+// Three variants of one kernel, chosen per call by the host; all take 64-key blocks.
 //   V = 0: d_R = 64: 4 K/V stages, separate exchange and P buffers; a warpgroup hands its
 //          exchange buffer back to the peer as soon as it has read it.
 //   V = 1: d_R = 512 (the wide positional key): each CTA's 256 RoPE dims as four 64-dim
 //          boxes, Q's RoPE half (64 KB) in shared memory, 2 K/V stages of 64 KB.  P is
 //          written over the exchange buffer once the scores are read, and the PV
 //          product's commit, multicast to the peer, hands the buffer back.
+//   V = 2: d_R = 64 over the low-bit ring: as V = 0, but no TMA fills the K/V stages.  Two
+//          warps read each block's packed codes and scales from global memory and write
+//          the dequantised bf16 rows into the stage in the layout the TMA loads would
+//          have, one key per lane (384 threads).
 // K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
 // swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of stage s at
 // OFF_KVR + (q * NST + s) * RBB.
@@ -71,6 +73,8 @@ constexpr int NTHREADS = 352;
 template <int V>
 struct Lay {
   static constexpr bool WIDE = V == 1;
+  static constexpr bool PACKED = V == 2;
+  static constexpr int NT = PACKED ? 384 : 352;              // threads
   static constexpr int NST = WIDE ? 2 : 4;
   static constexpr bool MERGED = WIDE;
   static constexpr int BNK = 64;                             // keys per block
@@ -228,8 +232,43 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, uint32_t tq, int64_t g
   tmem_wait_st();
 }
 
+// Dequantise one key's packed row of this CTA's half into K/V stage rows (one lane = one
+// key row k of the block).  A code pair becomes the bf16 pair (bias + c0, bias + c1) by
+// placing the biased fields in the low mantissa bits of 128.0 (exact), then c = that - bias
+// (exact) and c * s with s the row's scale rounded to bf16: one rounding of the product to
+// bf16, as the MMA operand needs.
+__device__ __forceinline__ uint32_t dq_pair(uint32_t biased_pair, uint32_t bias2, uint32_t s2) {
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&biased_pair);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&bias2);
+  const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&s2);
+  v = __hmul2(__hsub2(v, b), sc);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// eight INT4 codes (one 32-bit word, code i at bits 4i) -> eight bf16 (one 16-byte chunk)
+__device__ __forceinline__ uint4 dq8_int4(uint32_t w, uint32_t s2) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;   // codes 2k, 2k+1 in byte k
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    // byte k of lo to bits 0-7, byte k of hi to bits 16-23; then 0x4300 | (code ^ 8)
+    const uint32_t pr = __byte_perm(lo, hi, (uint32_t)(k | (k << 4) | ((k + 4) << 8) | ((k + 4) << 12)));
+    o[k] = dq_pair((pr & 0x000F000Fu) ^ 0x43084308u, 0x43084308u, s2);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+// eight INT2 codes (the low 16 bits of w, code i at bits 2i) -> eight bf16
+__device__ __forceinline__ uint4 dq8_int2(uint32_t w, uint32_t s2) {
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t f = (w >> (4 * k)) & 0xFu;               // codes 2k (bits 0-1), 2k+1 (2-3)
+    o[k] = dq_pair(((f & 3u) | ((f >> 2) << 16)) ^ 0x43024302u, 0x43024302u, s2);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 template <int V>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
                   const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ AttnArgs a,
                   const __grid_constant__ Sched sc) {
@@ -257,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&bar[B_KVF + s], 1);
+      mbar_init(&bar[B_KVF + s], LY::PACKED ? 64 : 1);   // TMA, or the two dequantising warps
       mbar_init(&bar[B_KVE + s], 1);
       mbar_init(&bar[B_KRE + s], 1);
     }
@@ -291,7 +330,89 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   SegWalk sw;
   sw.begin(sc, a, blockIdx.x >> 1);
 
-  if (warp == 8) {
+  if (LY::PACKED && (warp == 8 || warp == 11)) {
+    // ------------------------------------------------------------ dequantising producers
+    // Lane `lane` of warp 8 fills key row `lane` of every block's stage, warp 11 row
+    // 32 + lane.  Its packed codes are loaded before the wait for the stage, so their
+    // latency overlaps it; the blocks two ahead are asked into L2 meanwhile.
+    const int kr = (warp == 8 ? 0 : 32) + lane;
+    // content codes of 4 or 2 bits, RoPE codes of 4 bits (the host checks)
+    const int cb = a.cbits;
+    const int64_t crow = (int64_t)G.Dc * cb / 8, rrow = (int64_t)G.Dr / 2;
+    const int chalf = HALF * cb / 8, rhalf = LY::RHALF / 2;       // this CTA's bytes of a row
+    bool ok = true;
+    for (; ok && sw.valid(); sw.next(a)) {
+      for (int j = sw.jb; j < sw.je; ++j) {
+        const int g = sw.gbase + (j - sw.jb);
+        const int s = g % NST;
+        const uint32_t fph = ((g / NST) & 1) ^ 1;
+        int64_t slot0, g0;
+        int valid;
+        sw.tg.blk.get(j, slot0, g0, valid);
+        if (j + 2 < sw.je) {
+          int64_t s2_, g2_;
+          int v2_;
+          sw.tg.blk.get(j + 2, s2_, g2_, v2_);
+          if (kr < v2_) {
+            const int64_t row2 = (int64_t)sw.tg.b * G.S + s2_ + kr;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.pk_c + row2 * crow + rank * chalf));
+          }
+        }
+        const bool live = kr < valid;
+        const int64_t row = (int64_t)sw.tg.b * G.S + slot0 + kr;
+        uint4 cw[8];
+        uint4 rw = make_uint4(0, 0, 0, 0);
+        float scc = 0.f, scr = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cw[q] = make_uint4(0, 0, 0, 0);
+        if (live) {
+          const uint4* pc = reinterpret_cast<const uint4*>(a.pk_c + row * crow + rank * chalf);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q < chalf / 16) cw[q] = __ldg(pc + q);
+          rw = __ldg(reinterpret_cast<const uint4*>(a.pk_r + row * rrow + rank * rhalf));
+          scc = __ldg(a.sc_c + row);
+          scr = __ldg(a.sc_r + row);
+        }
+        ok = mbar_wait(&bar[B_KVE + s], fph, abort, a.err, 0x109, (kr << 16) | j);
+        if (!ok) break;
+        const uint32_t s2c = pack_bf16(scc, scc), s2r = pack_bf16(scr, scr);
+        // the four 64-dim latent boxes: row kr, 16-byte chunk c at chunk c ^ (kr % 8)
+#pragma unroll
+        for (int bq = 0; bq < 4; ++bq) {
+          uint8_t* box = sm + OFF_KV + (bq * NST + s) * BOX_BYTES + kr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int e = bq * 64 + c * 8;                      // first dim of the chunk
+            uint4 v;
+            if (cb == 4) {
+              const uint4 w4 = cw[e / 32];
+              const uint32_t w = ((e / 8) & 3) == 0 ? w4.x : ((e / 8) & 3) == 1 ? w4.y
+                                 : ((e / 8) & 3) == 2 ? w4.z : w4.w;
+              v = dq8_int4(w, s2c);
+            } else {
+              const uint4 w4 = cw[e / 64];
+              const int h = (e / 8) & 7;                          // 16-bit half of the uint4
+              const uint32_t w32 = (h >> 1) == 0 ? w4.x : (h >> 1) == 1 ? w4.y
+                                   : (h >> 1) == 2 ? w4.z : w4.w;
+              v = dq8_int2((h & 1) ? (w32 >> 16) : (w32 & 0xFFFFu), s2c);
+            }
+            *reinterpret_cast<uint4*>(box + ((c ^ (kr & 7)) * 16)) = v;
+          }
+        }
+        // the 32-dim RoPE box (64-byte rows, 64-byte swizzle: chunk c at c ^ ((kr / 2) % 4))
+        {
+          uint8_t* box = sm + OFF_KVR + s * RBOX_BYTES + kr * 64;
+          const uint32_t rws[4] = {rw.x, rw.y, rw.z, rw.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(box + ((c ^ ((kr >> 1) & 3)) * 16)) = dq8_int4(rws[c], s2r);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bar[B_KVF + s]);
+      }
+    }
+  } else if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
@@ -848,7 +969,7 @@ int cluster_slots() {
   // uses the smallest count any of them reaches
   int n = MAXC;
   bool ok = true;
-  auto probe = [&](auto kern, int smem) {
+  auto probe = [&](auto kern, int smem, int threads) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess) {
       ok = false;
@@ -856,14 +977,15 @@ int cluster_slots() {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * MAXC);
-    cfg.blockDim = dim3(NTHREADS);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     int c = 0;
     if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) != cudaSuccess || c < 1) c = 0;
     n = c < n ? c : n;
   };
-  probe(attend_kernel<0>, Lay<0>::SMEM);
-  probe(attend_kernel<1>, Lay<1>::SMEM);
+  probe(attend_kernel<0>, Lay<0>::SMEM, Lay<0>::NT);
+  probe(attend_kernel<1>, Lay<1>::SMEM, Lay<1>::NT);
+  probe(attend_kernel<2>, Lay<2>::SMEM, Lay<2>::NT);
   if (!ok) return 0;
   if (n < 1) {
     int sms = 0;
@@ -888,15 +1010,30 @@ bool tc_attend_supported(const Geo& g) {
 size_t tc_attend_workspace(const Geo& g) { return 2 * (size_t)cluster_slots() * slot_bytes(g); }
 
 
+bool tc_attend_packed_supported(const Geo& g, int cbits, int rbits) {
+  return g.Dc == 2 * HALF && g.Dr == 2 * Lay<2>::RHALF && (cbits == 4 || cbits == 2) &&
+         rbits == 4;
+}
+
 cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
                       const void* cache, int64_t k_first, int64_t n_keys, float scale,
                       void* o_lat, float* lse, void* workspace, size_t workspace_bytes,
                       unsigned int* err, cudaStream_t st) {
+  return tc_attend_ring(g, q_abs, n_q, q_first, cache, nullptr, k_first, n_keys, scale, o_lat,
+                        lse, workspace, workspace_bytes, err, st);
+}
+
+cudaError_t tc_attend_ring(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_first,
+                           const void* cache, const PackedRing* pk, int64_t k_first,
+                           int64_t n_keys, float scale, void* o_lat, float* lse,
+                           void* workspace, size_t workspace_bytes, unsigned int* err,
+                           cudaStream_t st) {
   const int tiles_per_batch = (int)((n_q * g.H + TM - 1) / TM);
-  const int variant = g.Dr == 2 * Lay<1>::RHALF ? 1 : 0;      // the wide positional key
+  // the low-bit ring, the wide positional key, or d_R = 64
+  const int variant = pk ? 2 : (g.Dr == 2 * Lay<1>::RHALF ? 1 : 0);
   const int bn = variant == 1 ? Lay<1>::BNK : Lay<0>::BNK;
-  CUtensorMap K, KR, QR;
-  {
+  CUtensorMap K{}, KR{}, QR;
+  if (!pk) {
     // K: 64-dim boxes of bn cached rows (the latent boxes, and the wide RoPE boxes);
     // KR: the 32-dim RoPE box of d_R = 64 (64-byte swizzle)
     uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.S, (uint64_t)g.B};
@@ -936,7 +1073,15 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
   a.bn = bn;
   // a sequence's keys are read by its tiles only: with one or two tiles (decode) each key
   // block comes from HBM once, and the producer looks PF_BLOCKS blocks ahead
-  a.pf = tiles_per_batch <= 2 ? PF_BLOCKS : 0;
+  a.pf = !pk && tiles_per_batch <= 2 ? PF_BLOCKS : 0;
+  if (pk) {
+    a.pk_c = static_cast<const uint8_t*>(pk->codes_c);
+    a.pk_r = static_cast<const uint8_t*>(pk->codes_r);
+    a.sc_c = pk->scale_c;
+    a.sc_r = pk->scale_r;
+    a.cbits = pk->cbits;
+    a.rbits = pk->rbits;
+  }
   a.err = err;
   const bool split = workspace != nullptr && workspace_bytes >= tc_attend_workspace(g);
 
@@ -952,7 +1097,9 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     int dev = 0, l2 = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) == cudaSuccess && l2 > 0) {
-      const double keys_bytes = (double)n_keys * g.row * 2;     // one sequence's keys
+      const double key_bytes = pk ? (double)g.Dc * pk->cbits / 8 + g.Dr * pk->rbits / 8 + 8
+                                  : (double)g.row * 2;
+      const double keys_bytes = (double)n_keys * key_bytes;     // one sequence's keys
       if (keys_bytes * g.B > l2 / 3.0) {
         const int by_l2 = (int)((l2 / 3.0) / keys_bytes);                  // fit a third of L2
         const int fill = (4 * ncl + tiles_per_batch - 1) / tiles_per_batch;   // >= 4 tiles each
@@ -1075,10 +1222,12 @@ cudaError_t tc_attend(const Geo& g, const void* q_abs, int64_t n_q, int64_t q_fi
     a.ws_lse = reinterpret_cast<float*>(a.ws_o + (size_t)2 * ncl * TM * g.Dc);
   }
   for (const Plan& p : plans) {
-    if (variant == 1)
-      attend_kernel<1><<<(unsigned)(2 * p.G), NTHREADS, Lay<1>::SMEM, st>>>(K, KR, QR, a, p.sc);
+    if (variant == 2)
+      attend_kernel<2><<<(unsigned)(2 * p.G), Lay<2>::NT, Lay<2>::SMEM, st>>>(K, KR, QR, a, p.sc);
+    else if (variant == 1)
+      attend_kernel<1><<<(unsigned)(2 * p.G), Lay<1>::NT, Lay<1>::SMEM, st>>>(K, KR, QR, a, p.sc);
     else
-      attend_kernel<0><<<(unsigned)(2 * p.G), NTHREADS, Lay<0>::SMEM, st>>>(K, KR, QR, a, p.sc);
+      attend_kernel<0><<<(unsigned)(2 * p.G), Lay<0>::NT, Lay<0>::SMEM, st>>>(K, KR, QR, a, p.sc);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);

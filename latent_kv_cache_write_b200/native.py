@@ -44,6 +44,8 @@ SIGNATURES = {
     "mla_cache_shift_frames": (_i32, [_P, _vp, _i64, _i64, _i64, _vp]),
     "mla_cache_quantise": (_i32, [_P, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "mla_cache_dequantise": (_i32, [_P, _vp, _vp, _vp, _vp, _i32, _i32, _i64, _i64, _vp, _vp]),
+    "mla_attend_quantised": (_i32, [_P, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _i64,
+                                    _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "mla_attend_materialised_workspace_size": (_sz, [_P]),
     "mla_attend_materialised": (_i32, [_P, _vp, _vp, _i64, _i64, _vp, _i64, _i64, _f32, _vp, _vp,
                                        _vp, _vp, _vp, _sz, _vp]),

@@ -257,3 +257,25 @@ def test_fixed_scratch_validation(L):
     assert _fixed(L, s, n_q=0) == native.MLA_OK               # empty: nothing to do
     big = _shape(batch=1000, n_heads=65, ring_slots=50000)
     assert _fixed(L, big, n_q=40000, q_first=0, n_keys=50000) == native.MLA_ERR_UNSUPPORTED
+
+
+def test_attend_quantised_validation(L):
+    s = _shape()
+
+    def aq(shape=s, q=FAKE, qc=FAKE, qr=FAKE, sc=FAKE, sr=FAKE, cb=4, rb=4, n_q=1560,
+           q_first=3 * 1560, k_first=0, n_keys=6240, o=FAKE, ws=None, ws_bytes=0):
+        return L.mla_attend_quantised(ctypes.byref(shape), q, n_q, q_first, qc, qr, sc, sr, cb,
+                                      rb, k_first, n_keys, 0.07, o, None, ws, ws_bytes, None)
+
+    A, U = native.MLA_ERR_ARG, native.MLA_ERR_UNSUPPORTED
+    for name in ("q", "qc", "qr", "sc", "sr", "o"):
+        assert aq(**{name: None}) == A, name
+    for name in ("q", "qr", "sc", "sr", "o"):
+        assert aq(**{name: ODD}) == native.MLA_ERR_ALIGN, name
+    assert aq(cb=3) == A and aq(rb=5) == A              # not a code width at all
+    assert aq(cb=8) == U and aq(rb=2) == U and aq(rb=8) == U    # widths the kernel lacks
+    assert aq(shape=_shape(dtype=native.MLA_F32)) == U
+    assert aq(shape=native.make_shape(C.WIDE_KEY), q_first=9 * 1560, n_keys=15600) == U
+    assert aq(n_keys=6241) == native.MLA_ERR_RANGE
+    assert aq(q_first=3 * 1560 + 1) == native.MLA_ERR_RANGE
+    assert aq(n_q=0, q_first=0) == native.MLA_OK

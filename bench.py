@@ -37,6 +37,7 @@ from synth import generate as G  # noqa: E402
 WORKLOAD = C.VIDEO_CHUNK            # the default step; --workload picks another
 # workloads whose step writes its own cache (decode reads a cache given directly and is
 # timed by the decode leg)
+LEGS = ("decode", "materialised", "shift", "quant", "fold", "quant_attend", "workloads")
 STEP_WORKLOADS = tuple(w.name for w in C.ALL if not w.cache_direct and w.elem_bytes == 2)
 L2_FLUSH_BYTES = 256 << 20           # > 126 MB L2: written between timed steps
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -550,6 +551,67 @@ def quant_attend_leg(torch, mla, steps, warmup, flush, peaks, chunk_step=None):
     return out
 
 
+def fold_leg(torch, mla, steps, warmup, flush, chunk_step=None):
+    """Whether to fold W_UV into the output projection ("Multi-Head Latent Attention" concept
+    page, "Low-rank joint compression": the same trick folds W^UV into the output
+    projection).  The pages give no output projection; W_O is taken as [n_h d_h, d] with the
+    hidden width d = 4096.  Two forms of y = concat_h(W_UV[h] o_lat[h]) W_O, both timed with
+    the L2 flushed: mla_up_v and then the W_O GEMM, against one GEMM with the folded weight
+    [n_h d_c, d] (W_UV[h]^T W_O[h] stacked over heads).  Both W_O GEMMs are cuBLAS calls
+    (torch.matmul), as a measurement: the projection is not part of the path."""
+    res = {}
+    d = 4096
+    dev = "cuda"
+    cases = []
+    wl = C.DECODE
+    shape = mla.make_shape(wl)
+    g = torch.Generator(device=dev).manual_seed(0)
+    o_lat = (torch.randn((wl.batch, 1, wl.n_heads, wl.d_latent), device=dev, generator=g)
+             .to(torch.bfloat16))
+    w_uv = (torch.randn((wl.n_heads, wl.d_nope, wl.d_latent), device=dev, generator=g)
+            / wl.d_latent ** 0.5).to(torch.bfloat16)
+    cases.append(("decode", wl, shape, o_lat, w_uv, 1))
+    if chunk_step is not None:
+        st = chunk_step
+        cases.append(("video_chunk", st.wl, st.shape, st.o_lat, st.w["w_uv"], st.wl.n_queries))
+    for name, wl, shape, o_lat, w_uv, T in cases:
+        H, dh, dc = wl.n_heads, wl.d_nope, wl.d_latent
+        w_o = (torch.randn((H * dh, d), device=dev, generator=g) / (H * dh) ** 0.5).to(torch.bfloat16)
+        # folded weight: rows h*dc .. h*dc+dc-1 = W_UV[h]^T W_O[h*dh : (h+1)*dh]
+        w_fold = torch.einsum("hkc,hkd->hcd", w_uv.float(), w_o.view(H, dh, d).float()) \
+            .reshape(H * dc, d).to(torch.bfloat16)
+        out = torch.empty((wl.batch, T, H, dh), dtype=torch.bfloat16, device=dev)
+        rows = wl.batch * T
+
+        def two_step(_a=None):
+            mla.mla_up_v(shape, o_lat, T, w_uv, out)
+            return out.view(rows, H * dh) @ w_o
+
+        def folded(_a=None):
+            return o_lat.view(rows, H * dc) @ w_fold
+
+        y2, y1 = two_step(), folded()
+        torch.cuda.synchronize()
+        rel = float((y1.float() - y2.float()).norm() / y2.float().norm())
+        for _ in range(warmup):
+            two_step()
+            folded()
+        ms2, _ = time_steps(torch, two_step, steps, flush)
+        ms1, _ = time_steps(torch, folded, steps, flush)
+        res[name] = {"rows": rows, "two_step_ms": statistics.mean(ms2),
+                     "folded_ms": statistics.mean(ms1),
+                     "folded_over_two_step": statistics.mean(ms1) / statistics.mean(ms2),
+                     "weight_bytes_two_step": int((w_uv.numel() + w_o.numel()) * 2),
+                     "weight_bytes_folded": int(w_fold.numel() * 2),
+                     "flops_two_step": 2 * rows * H * dc * dh + 2 * rows * H * dh * d,
+                     "flops_folded": 2 * rows * H * dc * d,
+                     "rel_diff": rel}
+        del w_fold, w_o
+    res["note"] = ("W_O [n_h d_h, 4096] assumed (the pages give none); both W_O GEMMs are "
+                   "cuBLAS; the folded weight is d_c / d_h = 4x the size of W_O")
+    return res
+
+
 _CPU_STATE = {}
 
 
@@ -710,7 +772,12 @@ def run_ours(args):
     att_ms = kernels_ms["attend"]
     achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    dec = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush) if rank == 0 else None
+    legs = set(LEGS) if args.legs == "all" else set(args.legs.split(","))
+    unknown = legs - set(LEGS)
+    if unknown:
+        raise SystemExit(f"unknown legs: {sorted(unknown)}")
+    leg = lambda name: rank == 0 and name in legs
+    dec = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush) if leg("decode") else None
     if dec:
         # small-batch decode: one sequence, its keys split over every cluster
         one = decode_leg(torch, mla, max(3, args.steps), args.warmup, flush,
@@ -719,23 +786,25 @@ def run_ours(args):
                                "bytes": one["bytes"]}
     mat = materialised_leg(torch, mla, step, max(3, args.steps), args.warmup, flush,
                            kernels_ms["absorb_q"] + kernels_ms["attend"] + kernels_ms["up_v"]) \
-        if rank == 0 else None
+        if leg("materialised") else None
     if mat:
         mat["frac"] = mat["tflops"] / float(peaks["bf16_tflops"])
     shift = shift_leg(torch, mla, step, max(3, args.steps), args.warmup, flush) \
-        if rank == 0 else None
+        if leg("shift") else None
     quant = quant_leg(torch, mla, step, max(3, args.steps), args.warmup, flush) \
-        if rank == 0 else None
+        if leg("quant") else None
     if dec:
         dec["peak_gbs"] = float(peaks["hbm_gbs"])
         dec["frac"] = dec["value"] / dec["peak_gbs"]
+    fold = fold_leg(torch, mla, max(3, args.steps), args.warmup, flush, step) \
+        if leg("fold") else None
     qatt = quant_attend_leg(torch, mla, max(3, args.steps), args.warmup, flush, peaks, step) \
-        if rank == 0 else None
+        if leg("quant_attend") else None
     # the long-window and wide-positional-key steps, in the same run
     others = {n: workload_leg(torch, mla, n, max(3, min(args.steps, 10)), args.warmup, flush,
                               peaks, local)
               for n in ("long_window_bf16", "wide_key_bf16") if n != wl.name} \
-        if rank == 0 else None
+        if leg("workloads") else None
     if rank == 0:
         line = {
             "metric": "absorbed MLA attention TFLOP/s (chunk) and latent-cache GB/s (decode) "
@@ -769,6 +838,7 @@ def run_ours(args):
             "k_rope_shift": shift,
             "quant_ring": quant,
             "quant_attend": qatt,
+            "fold_w_uv_into_w_o": fold,
             "workloads": others,
             "clocks": clocks.summary(),
             "kernels_ms": kernels_ms,
@@ -833,6 +903,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD.name, choices=STEP_WORKLOADS,
                     help="the step's workload (default: the video chunk)")
+    ap.add_argument("--legs", default="all",
+                    help="comma-separated extra legs to run after the step (default all: "
+                         + ",".join(LEGS) + "); fewer legs make a shorter run to profile")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

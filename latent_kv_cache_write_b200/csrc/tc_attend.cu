@@ -61,10 +61,10 @@ using namespace attn;
 //          boxes, Q's RoPE half (64 KB) in shared memory, 2 K/V stages of 64 KB.  P is
 //          written over the exchange buffer once the scores are read, and the PV
 //          product's commit, multicast to the peer, hands the buffer back.
-//   V = 2: d_R = 64 over the low-bit ring: as V = 0, but no TMA fills the K/V stages.  Two
-//          warps read each block's packed codes and scales from global memory and write
-//          the dequantised bf16 rows into the stage in the layout the TMA loads would
-//          have, one key per lane (384 threads).
+//   V = 2: d_R = 64 over the low-bit ring: as V = 0 with 3 K/V stages, and the stages are
+//          not loaded but written.  TMA brings each block's packed codes and scales into a
+//          3-slot staging ring, and two warps (one key row per lane; 384 threads) write the
+//          dequantised bf16 rows into the stage in the layout the TMA loads would have.
 // K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
 // swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of stage s at
 // OFF_KVR + (q * NST + s) * RBB.
@@ -75,7 +75,7 @@ struct Lay {
   static constexpr bool WIDE = V == 1;
   static constexpr bool PACKED = V == 2;
   static constexpr int NT = PACKED ? 384 : 352;              // threads
-  static constexpr int NST = WIDE ? 2 : 4;
+  static constexpr int NST = WIDE ? 2 : (PACKED ? 3 : 4);
   static constexpr bool MERGED = WIDE;
   static constexpr int BNK = 64;                             // keys per block
   static constexpr int BOXB = BNK * 64 * 2;                  // latent box: BNK keys x 64 dims
@@ -89,7 +89,15 @@ struct Lay {
   static constexpr int XPB = TM * BNK * 2;                   // exchange / P buffer (128-byte rows)
   static constexpr int OFF_KV = 0;
   static constexpr int OFF_KVR = OFF_KV + NST * LATB;
-  static constexpr int OFF_QR = OFF_KVR + NST * NRB * RBB;
+  // packed variant: staging slots of one block's codes (this CTA's half of 64 rows; content
+  // slots 1024-byte aligned for the swizzle) and scales (68 floats from a 16-byte aligned
+  // row, per path)
+  static constexpr int NSG = PACKED ? 3 : 0;
+  static constexpr int SGC = 64 * 128, SGR = 64 * 16, SGS = 2 * 384;   // 128-byte aligned boxes
+  static constexpr int OFF_SG = OFF_KVR + NST * NRB * RBB;          // content [NSG]
+  static constexpr int OFF_SGR = OFF_SG + NSG * SGC;                // RoPE codes [NSG]
+  static constexpr int OFF_SGS = OFF_SGR + NSG * SGR;               // scales [NSG]
+  static constexpr int OFF_QR = (OFF_SGS + NSG * SGS + 1023) / 1024 * 1024;
   static constexpr int OFF_X = OFF_QR + QRB;                 // [2] exchange buffers
   static constexpr int OFF_P = MERGED ? OFF_X : OFF_X + 2 * XPB;   // [2] P buffers
   static constexpr int OFF_M = OFF_P + 2 * XPB;              // running max [2][128]
@@ -110,10 +118,15 @@ struct Lay {
   static constexpr int B_M = B_PE + 2;          // running max of a block published (128) [2]
   static constexpr int B_KRE = B_M + 2;         // RoPE boxes of a stage free (wide; MMA commit
                                                 // after the scores)                      [NST]
-  static constexpr int NBAR = B_KRE + NST;
+  static constexpr int B_SGF = B_KRE + NST;    // staging slot loaded (TMA)           [NSG]
+  static constexpr int B_SGE = B_SGF + NSG;    // staging slot read (64)               [NSG]
+  static constexpr int NBAR = B_SGE + NSG;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 48 + 1024;   // TMEM slot, abort flag, votes [2][4]
   static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
+  static_assert(OFF_SG % 1024 == 0 && OFF_SGR % 128 == 0 && OFF_SGS % 128 == 0 &&
+                OFF_QR % 1024 == 0 && OFF_X % 1024 == 0 && OFF_P % 1024 == 0,
+                "TMA and swizzled boxes start on their alignment");
 };
 
 constexpr uint32_t O_COL = 0, Q_COL = 256, S_COL = 384;
@@ -270,7 +283,8 @@ __device__ __forceinline__ uint4 dq8_int2(uint32_t w, uint32_t s2) {
 template <int V>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
-                  const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ AttnArgs a,
+                  const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ CUtensorMap tmSC,
+                  const __grid_constant__ CUtensorMap tmSR, const __grid_constant__ AttnArgs a,
                   const __grid_constant__ Sched sc) {
   using LY = Lay<V>;
   constexpr int NST = LY::NST;
@@ -299,6 +313,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
       mbar_init(&bar[B_KVF + s], LY::PACKED ? 64 : 1);   // TMA, or the two dequantising warps
       mbar_init(&bar[B_KVE + s], 1);
       mbar_init(&bar[B_KRE + s], 1);
+    }
+    for (int q = 0; q < LY::NSG; ++q) {
+      mbar_init(&bar[LY::B_SGF + q], 1);
+      mbar_init(&bar[LY::B_SGE + q], 64);
     }
     mbar_init(&bar[B_QR], 1);
     mbar_init(&bar[B_QREADY], 256);
@@ -332,84 +350,113 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
 
   if (LY::PACKED && (warp == 8 || warp == 11)) {
     // ------------------------------------------------------------ dequantising producers
-    // Lane `lane` of warp 8 fills key row `lane` of every block's stage, warp 11 row
-    // 32 + lane.  Its packed codes are loaded before the wait for the stage, so their
-    // latency overlaps it; the blocks two ahead are asked into L2 meanwhile.
+    // Lane 0 of warp 8 keeps the staging ring NSG blocks ahead with TMA: the block's
+    // content codes (this CTA's half of 64 rows, 128- or 64-byte swizzle), its RoPE codes and
+    // both paths' scales.  Lane `lane` of warp 8 turns key row `lane` of every block into
+    // bf16 stage rows, warp 11 row 32 + lane.
+    constexpr int NSG = LY::NSG > 0 ? LY::NSG : 1;   // (the branch is dead for V = 0, 1)
     const int kr = (warp == 8 ? 0 : 32) + lane;
-    // content codes of 4 or 2 bits, RoPE codes of 4 bits (the host checks)
-    const int cb = a.cbits;
-    const int64_t crow = (int64_t)G.Dc * cb / 8, rrow = (int64_t)G.Dr / 2;
-    const int chalf = HALF * cb / 8, rhalf = LY::RHALF / 2;       // this CTA's bytes of a row
+    const int cb = a.cbits;                       // 4 or 2; RoPE codes are 4 bits
+    const int chalf = HALF * cb / 8;              // content bytes of a row for this CTA
+    const bool issuer = warp == 8 && lane == 0;
+    SegWalk iw = sw;                              // the issuer's walk, NSG blocks ahead
+    int ij = iw.valid() ? iw.jb : 0, issued = 0;
+    auto issue_next = [&]() -> bool {
+      if (!iw.valid()) return true;
+      const int q = issued % NSG;
+      if (!mbar_wait(&bar[LY::B_SGE + q], ((issued / NSG) & 1) ^ 1, abort, a.err, 0x10B, issued))
+        return false;
+      int64_t slot0, g0;
+      int valid;
+      iw.tg.blk.get(ij, slot0, g0, valid);
+      const int32_t row0 = (int32_t)((int64_t)iw.tg.b * G.S + slot0);
+      const int32_t row4 = row0 & ~3;             // scales from a 16-byte aligned element
+      uint8_t* scl = sm + LY::OFF_SGS + q * LY::SGS;
+      mbar_expect_tx(&bar[LY::B_SGF + q], 64 * chalf + LY::SGR + 2 * 68 * 4);
+      tma_load_2d(sm + LY::OFF_SG + q * LY::SGC, &tmK, &bar[LY::B_SGF + q], (int)rank * chalf, row0);
+      tma_load_2d(sm + LY::OFF_SGR + q * LY::SGR, &tmKR, &bar[LY::B_SGF + q], (int)rank * 16, row0);
+      tma_load_1d(scl, &tmSC, &bar[LY::B_SGF + q], row4);
+      tma_load_1d(scl + 384, &tmSR, &bar[LY::B_SGF + q], row4);
+      ++issued;
+      if (++ij >= iw.je) {
+        iw.next(a);
+        ij = iw.valid() ? iw.jb : 0;
+      }
+      return true;
+    };
     bool ok = true;
+    if (issuer) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmKR);
+      prefetch_tmap(&tmSC);
+      prefetch_tmap(&tmSR);
+      for (int q = 0; ok && q < NSG; ++q) ok = issue_next();
+    }
     for (; ok && sw.valid(); sw.next(a)) {
       for (int j = sw.jb; j < sw.je; ++j) {
         const int g = sw.gbase + (j - sw.jb);
-        const int s = g % NST;
-        const uint32_t fph = ((g / NST) & 1) ^ 1;
+        const int s = g % NST, q = g % NSG;
         int64_t slot0, g0;
         int valid;
         sw.tg.blk.get(j, slot0, g0, valid);
-        if (j + 2 < sw.je) {
-          int64_t s2_, g2_;
-          int v2_;
-          sw.tg.blk.get(j + 2, s2_, g2_, v2_);
-          if (kr < v2_) {
-            const int64_t row2 = (int64_t)sw.tg.b * G.S + s2_ + kr;
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.pk_c + row2 * crow + rank * chalf));
-          }
-        }
-        const bool live = kr < valid;
-        const int64_t row = (int64_t)sw.tg.b * G.S + slot0 + kr;
-        uint4 cw[8];
-        uint4 rw = make_uint4(0, 0, 0, 0);
-        float scc = 0.f, scr = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) cw[q] = make_uint4(0, 0, 0, 0);
-        if (live) {
-          const uint4* pc = reinterpret_cast<const uint4*>(a.pk_c + row * crow + rank * chalf);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (q < chalf / 16) cw[q] = __ldg(pc + q);
-          rw = __ldg(reinterpret_cast<const uint4*>(a.pk_r + row * rrow + rank * rhalf));
-          scc = __ldg(a.sc_c + row);
-          scr = __ldg(a.sc_r + row);
-        }
-        ok = mbar_wait(&bar[B_KVE + s], fph, abort, a.err, 0x109, (kr << 16) | j);
+        ok = mbar_wait(&bar[LY::B_SGF + q], (g / NSG) & 1, abort, a.err, 0x10A, (kr << 16) | j);
+        if (ok) ok = mbar_wait(&bar[B_KVE + s], ((g / NST) & 1) ^ 1, abort, a.err, 0x109,
+                               (kr << 16) | j);
         if (!ok) break;
+        const uint8_t* scl = sm + LY::OFF_SGS + q * LY::SGS;
+        const bool live = kr < valid;
+        const int r4 = (int)(((int64_t)sw.tg.b * G.S + slot0) & 3) + kr;   // scale index
+        const float scc = live ? reinterpret_cast<const float*>(scl)[r4] : 0.f;
+        const float scr = live ? reinterpret_cast<const float*>(scl + 384)[r4] : 0.f;
         const uint32_t s2c = pack_bf16(scc, scc), s2r = pack_bf16(scr, scr);
-        // the four 64-dim latent boxes: row kr, 16-byte chunk c at chunk c ^ (kr % 8)
-#pragma unroll
+        // this row's codes in the staging slot: 16-byte chunk c of a 128-byte row at chunk
+        // c ^ (kr % 8) (INT4), of a 64-byte row at c ^ ((kr / 2) % 4) (INT2)
+        const uint8_t* crow = sm + LY::OFF_SG + q * LY::SGC + kr * chalf;
+        // the four 64-dim latent boxes, one per iteration (a compact loop: the unrolled body
+        // would crowd the instruction cache the softmax warps share); row kr, 16-byte chunk c
+        // at chunk c ^ (kr % 8)
+#pragma unroll 1
         for (int bq = 0; bq < 4; ++bq) {
           uint8_t* box = sm + OFF_KV + (bq * NST + s) * BOX_BYTES + kr * 128;
+          uint32_t ww[8];
+          if (cb == 4) {
+            // box bq holds codes 64 bq .. 64 bq + 63: staging chunks 2 bq, 2 bq + 1
+            const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2 * bq) ^ (kr & 7)) * 16));
+            const uint4 c1 =
+                *reinterpret_cast<const uint4*>(crow + (((2 * bq + 1) ^ (kr & 7)) * 16));
+            ww[0] = c0.x; ww[1] = c0.y; ww[2] = c0.z; ww[3] = c0.w;
+            ww[4] = c1.x; ww[5] = c1.y; ww[6] = c1.z; ww[7] = c1.w;
+          } else {
+            const uint4 c0 = *reinterpret_cast<const uint4*>(crow + ((bq ^ ((kr >> 1) & 3)) * 16));
+            const uint32_t hw[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) ww[c] = (c & 1) ? (hw[c >> 1] >> 16) : (hw[c >> 1] & 0xFFFFu);
+          }
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const int e = bq * 64 + c * 8;                      // first dim of the chunk
-            uint4 v;
-            if (cb == 4) {
-              const uint4 w4 = cw[e / 32];
-              const uint32_t w = ((e / 8) & 3) == 0 ? w4.x : ((e / 8) & 3) == 1 ? w4.y
-                                 : ((e / 8) & 3) == 2 ? w4.z : w4.w;
-              v = dq8_int4(w, s2c);
-            } else {
-              const uint4 w4 = cw[e / 64];
-              const int h = (e / 8) & 7;                          // 16-bit half of the uint4
-              const uint32_t w32 = (h >> 1) == 0 ? w4.x : (h >> 1) == 1 ? w4.y
-                                   : (h >> 1) == 2 ? w4.z : w4.w;
-              v = dq8_int2((h & 1) ? (w32 >> 16) : (w32 & 0xFFFFu), s2c);
-            }
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (live) v = cb == 4 ? dq8_int4(ww[c], s2c) : dq8_int2(ww[c], s2c);
             *reinterpret_cast<uint4*>(box + ((c ^ (kr & 7)) * 16)) = v;
           }
         }
         // the 32-dim RoPE box (64-byte rows, 64-byte swizzle: chunk c at c ^ ((kr / 2) % 4))
         {
           uint8_t* box = sm + OFF_KVR + s * RBOX_BYTES + kr * 64;
+          const uint4 rw = *reinterpret_cast<const uint4*>(sm + LY::OFF_SGR + q * LY::SGR + kr * 16);
           const uint32_t rws[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(box + ((c ^ ((kr >> 1) & 3)) * 16)) = dq8_int4(rws[c], s2r);
+            *reinterpret_cast<uint4*>(box + ((c ^ ((kr >> 1) & 3)) * 16)) =
+                live ? dq8_int4(rws[c], s2r) : make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_KVF + s]);
+        mbar_arrive(&bar[LY::B_SGE + q]);          // the staging slot may be refilled
+        if (issuer) ok = issue_next();
+        if (!__all_sync(FULL, ok)) {
+          ok = false;
+          break;
+        }
       }
     }
   } else if (warp == 8) {
@@ -1032,8 +1079,34 @@ cudaError_t tc_attend_ring(const Geo& g, const void* q_abs, int64_t n_q, int64_t
   // the low-bit ring, the wide positional key, or d_R = 64
   const int variant = pk ? 2 : (g.Dr == 2 * Lay<1>::RHALF ? 1 : 0);
   const int bn = variant == 1 ? Lay<1>::BNK : Lay<0>::BNK;
-  CUtensorMap K{}, KR{}, QR;
-  if (!pk) {
+  CUtensorMap K{}, KR{}, QR, SC{}, SR{};
+  if (pk) {
+    // the packed ring: content codes (this CTA's half of a row per box row), RoPE codes,
+    // and the two paths' float32 scales
+    const uint64_t rows = (uint64_t)g.B * g.S;
+    const uint64_t crow = (uint64_t)g.Dc * pk->cbits / 8, rrow = (uint64_t)g.Dr * pk->rbits / 8;
+    const uint32_t chalf = (uint32_t)(crow / 2);
+    {
+      uint64_t d[2] = {crow, rows};
+      uint64_t st2[1] = {crow};
+      uint32_t b[2] = {chalf, 64};
+      if (!make_tmap_raw(&K, pk->codes_c, false, 2, d, st2, b, chalf == 128 ? 128 : 64))
+        return cudaErrorInvalidValue;
+    }
+    {
+      uint64_t d[2] = {rrow, rows};
+      uint64_t st2[1] = {rrow};
+      uint32_t b[2] = {(uint32_t)(rrow / 2), 64};
+      if (!make_tmap_raw(&KR, pk->codes_r, false, 2, d, st2, b, 0)) return cudaErrorInvalidValue;
+    }
+    {
+      uint64_t d[1] = {rows};
+      uint32_t b[1] = {68};
+      if (!make_tmap_raw(&SC, pk->scale_c, true, 1, d, nullptr, b, 0) ||
+          !make_tmap_raw(&SR, pk->scale_r, true, 1, d, nullptr, b, 0))
+        return cudaErrorInvalidValue;
+    }
+  } else {
     // K: 64-dim boxes of bn cached rows (the latent boxes, and the wide RoPE boxes);
     // KR: the 32-dim RoPE box of d_R = 64 (64-byte swizzle)
     uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.S, (uint64_t)g.B};
@@ -1223,11 +1296,11 @@ cudaError_t tc_attend_ring(const Geo& g, const void* q_abs, int64_t n_q, int64_t
   }
   for (const Plan& p : plans) {
     if (variant == 2)
-      attend_kernel<2><<<(unsigned)(2 * p.G), Lay<2>::NT, Lay<2>::SMEM, st>>>(K, KR, QR, a, p.sc);
+      attend_kernel<2><<<(unsigned)(2 * p.G), Lay<2>::NT, Lay<2>::SMEM, st>>>(K, KR, QR, SC, SR, a, p.sc);
     else if (variant == 1)
-      attend_kernel<1><<<(unsigned)(2 * p.G), Lay<1>::NT, Lay<1>::SMEM, st>>>(K, KR, QR, a, p.sc);
+      attend_kernel<1><<<(unsigned)(2 * p.G), Lay<1>::NT, Lay<1>::SMEM, st>>>(K, KR, QR, SC, SR, a, p.sc);
     else
-      attend_kernel<0><<<(unsigned)(2 * p.G), Lay<0>::NT, Lay<0>::SMEM, st>>>(K, KR, QR, a, p.sc);
+      attend_kernel<0><<<(unsigned)(2 * p.G), Lay<0>::NT, Lay<0>::SMEM, st>>>(K, KR, QR, SC, SR, a, p.sc);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);

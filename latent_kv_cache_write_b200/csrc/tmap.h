@@ -14,4 +14,9 @@ namespace mla {
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle64 = false);
 
+// uint8 (f32 false) or float32 tensor, otherwise as above; swizzle_bytes 0, 64 or 128.
+bool make_tmap_raw(CUtensorMap* map, const void* base, bool f32, int rank,
+                   const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                   int swizzle_bytes);
+
 }  // namespace mla

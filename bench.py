@@ -486,6 +486,11 @@ def workload_leg(torch, mla, name, steps, warmup, flush, peaks, device):
            "attend": {"ms": kms["attend"], "flops": fl["attend"], "tflops": att, "peak": peak,
                       "frac": att / peak, "p10_p50_p90": percentiles(dict(zip(Step.STAGES, parts))["attend"])},
            "kernels_ms": kms, "clocks": clocks.summary()}
+    mat = materialised_leg(torch, mla, step, steps, warmup, flush,
+                           kms["absorb_q"] + kms["attend"] + kms["up_v"])
+    if mat:
+        mat["frac"] = mat["tflops"] / peak
+        out["materialised"] = mat
     del step
     torch.cuda.empty_cache()
     return out

@@ -348,7 +348,7 @@ size_t mla_attend_materialised_workspace_size(const mla_shape* shape);
  *   lse    [B, n_q, n_h] float32 or NULL written
  *   workspace: at least mla_attend_materialised_workspace_size() bytes (required); its
  *   contents on entry do not matter, and calls sharing one must not run concurrently.
- * Supported: bf16 storage, d_nope = 128, d_rope = 64, d_latent a multiple of 128.
+ * Supported: bf16 storage, d_nope = 128, d_rope = 64 or 512, d_latent a multiple of 128.
  * Errors: those of mla_attend; MLA_ERR_UNSUPPORTED for other shapes or float32;
  * MLA_ERR_ARG if the workspace is NULL or smaller than required.
  */

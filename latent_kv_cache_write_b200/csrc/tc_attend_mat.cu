@@ -1,5 +1,5 @@
 // Non-absorbed ("materialised") MLA attention on tcgen05 tensor cores (bf16, d_nope = 128,
-// d_R = 64).
+// d_R = 64 or 512).
 //
 // The per-head keys and values are rebuilt from the latent beforehand for every ring slot
 // (tc_materialise: K_h = c . W_UK[h]^T and V_h = c . W_UV[h]^T, into the caller's
@@ -7,10 +7,11 @@
 // concatenation of the content and RoPE channels:
 //   s = scale * ([q_nope || RoPE(q_R)] . [K_h[slot] || k_R[slot]]),  o = softmax(s) . V_h.
 // A tile is 128 queries of one head, and one CTA holds it whole: O (128 x 128 fp32) and
-// the query (128 x 192 bf16) stay in TMEM beside two score buffers, so the CTAs share
-// nothing.  Per block of 64 keys the CTA
-//   - TMA-loads the block's K_h rows (two 64-dim boxes), its cached k_R rows (one box)
-//     and its V_h rows (two boxes),
+// the query (128 x (128 + d_R) bf16) stay in TMEM beside two score buffers, so the CTAs
+// share nothing.  Blocks are 64 keys for d_R = 64; for d_R = 512 the query takes 320 of the
+// 512 TMEM columns, so blocks are 32 keys (two 32-column score buffers).  Per block the CTA
+//   - TMA-loads the block's K_h rows (two 64-dim boxes), its cached k_R rows (one box, or
+//     eight for d_R = 512) and its V_h rows (two boxes),
 //   - computes S = Q . [K_h || k_R]^T with tcgen05.mma (the query as the TMEM A operand),
 //   - runs the online softmax of the 128 rows (two warpgroups take alternate blocks and
 //     hand each other the running row maximum),
@@ -37,21 +38,35 @@ using attn::key_end;
 using attn::TM;
 
 constexpr int NTHREADS = 352;
-constexpr int BN = 64;                         // keys per block
 constexpr int DN = 128;                        // d_nope: per-head key and value width
-constexpr int DR = 64;                         // d_R
 constexpr int NST = 4;                         // K/V ring stages
-constexpr int BOX = BN * 64 * 2;               // one 64-dim box of a block: 8 KB
-constexpr int STAGE = 5 * BOX;                 // K_h (2 boxes), k_R, V_h (2 boxes)
-constexpr int PBUF = TM * BN * 2;              // P of one block: 16 KB
-// ring, box-major: box q of stage s at OFF + (q * NST + s) * BOX
-constexpr int OFF_K = 0;
-constexpr int OFF_KR = OFF_K + 2 * NST * BOX;
-constexpr int OFF_V = OFF_KR + NST * BOX;
-constexpr int OFF_P = OFF_V + 2 * NST * BOX;   // [2]
-constexpr int OFF_M = OFF_P + 2 * PBUF;        // running max [2][128]
-constexpr int OFF_FREQ = OFF_M + 2 * TM * 4;   // RoPE frequencies [DR / 2] (double)
-constexpr int OFF_BAR = OFF_FREQ + DR / 2 * 8;
+
+// Layout of one variant (d_R = 64 or 512).  The ring is box-major: box q of stage s at
+// OFF + (q * NST + s) * BOX, a box being 64 dims of the block's BN rows (128-byte rows).
+template <int DRV>
+struct MLay {
+  static constexpr int DR = DRV;
+  static constexpr int BN = DRV == 512 ? 32 : 64;        // keys per block
+  static constexpr int BOX = BN * 64 * 2;                // one 64-dim box of a block
+  static constexpr int NRB = DR / 64;                    // k_R boxes per stage
+  static constexpr int STAGE = (4 + NRB) * BOX;          // K_h (2 boxes), k_R, V_h (2 boxes)
+  static constexpr int PBUF = TM * BN * 2;               // P of one block
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_KR = OFF_K + 2 * NST * BOX;
+  static constexpr int OFF_V = OFF_KR + NRB * NST * BOX;
+  static constexpr int OFF_P = OFF_V + 2 * NST * BOX;    // [2]
+  static constexpr int OFF_M = OFF_P + 2 * PBUF;         // running max [2][128]
+  static constexpr int OFF_FREQ = OFF_M + 2 * TM * 4;    // RoPE frequencies [DR / 2] (double)
+  static constexpr int OFF_BAR = OFF_FREQ + DR / 2 * 8;
+  static constexpr int NBAR = 4 * 2 + 4 + 10;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
+  static_assert(OFF_P % 1024 == 0, "P buffers on the swizzle atom");
+  // TMEM columns: O (128), the query (64 for q_nope + DR / 2 for the RoPE part), S [2]
+  static constexpr uint32_t O_COL = 0, Q_COL = 128, S_COL = DRV == 512 ? 448 : 256;
+  static_assert(S_COL + 2 * BN <= 512 && Q_COL + (DN + DR) / 2 <= S_COL, "TMEM columns");
+};
 constexpr int B_KVF = 0;                       // stage loaded (TMA)                   [NST]
 constexpr int B_KVE = B_KVF + NST;             // stage free (MMA commit after PV)    [NST]
 constexpr int B_QREADY = B_KVE + NST;          // the tile's query in TMEM (256)
@@ -63,12 +78,8 @@ constexpr int B_SE = B_SF + 2;                 // S buffer read (128)           
 constexpr int B_PF = B_SE + 2;                 // P written, O rescaled (128)          [2]
 constexpr int B_PE = B_PF + 2;                 // PV done (MMA commit)                 [2]
 constexpr int B_M = B_PE + 2;                  // running max of a block published (128) [2]
-constexpr int NBAR = B_M + 2;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM = OFF_MISC + 16 + 1024;
-static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
+static_assert(B_M + 2 == MLay<64>::NBAR, "barrier count");
 
-constexpr uint32_t O_COL = 0, Q_COL = 128, S_COL = 256;   // TMEM columns
 constexpr unsigned FULL = 0xffffffffu;
 
 struct MatArgs {
@@ -76,7 +87,7 @@ struct MatArgs {
   int64_t n_q, q_first, k_first, n_keys;
   float scale_log2;
   const bf16* q_nope;       // [B, n_q, H, DN]
-  const bf16* q_rope;       // [B, n_q, H, DR], un-rotated
+  const bf16* q_rope;       // [B, n_q, H, d_R], un-rotated
   bf16* out;                // [B, n_q, H, DN]
   float* lse;               // [B, n_q, H] or null
   int qblocks;              // 128-query blocks per (sequence, head)
@@ -91,6 +102,7 @@ struct MatTile {
   Blocks blk;
 };
 
+template <int BN>
 __device__ __forceinline__ MatTile mat_tile(const MatArgs& a, int t) {
   const Geo& G = a.g;
   MatTile m;
@@ -114,13 +126,14 @@ __device__ __forceinline__ MatTile mat_tile(const MatArgs& a, int t) {
 
 // The tiles of one CTA, in order, with the running counts that barrier phases and ring
 // stages derive from (every role walks the same sequence).
+template <int BN>
 struct TileWalk {
   int t, k, gbase, nbase0, nbase1;
   MatTile m;
   __device__ void begin(const MatArgs& a) {
     t = blockIdx.x;
     k = gbase = nbase0 = nbase1 = 0;
-    if (valid(a)) m = mat_tile(a, t);
+    if (valid(a)) m = mat_tile<BN>(a, t);
   }
   __device__ bool valid(const MatArgs& a) const { return t < a.tiles; }
   __device__ int nb() const { return m.blk.nblk; }
@@ -132,7 +145,7 @@ struct TileWalk {
     nbase1 += n >> 1;
     ++k;
     t += gridDim.x;
-    if (valid(a)) m = mat_tile(a, t);
+    if (valid(a)) m = mat_tile<BN>(a, t);
   }
 };
 
@@ -150,8 +163,9 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float f) {
 }
 
 // The query of row i of the tile into TMEM from column tq: warpgroup 0 writes q_nope
-// (64 columns of bf16 pairs), warpgroup 1 the RoPE'd q_R (32 columns), rotated by the
+// (64 columns of bf16 pairs), warpgroup 1 the RoPE'd q_R (DR / 2 columns), rotated by the
 // query token's (t, y, x) position.
+template <int DR>
 __device__ __forceinline__ void load_q(const MatArgs& a, const MatTile& m, uint32_t tq,
                                        int t, int wg, const double* inv_freq) {
   const Geo& G = a.g;
@@ -175,16 +189,17 @@ __device__ __forceinline__ void load_q(const MatArgs& a, const MatTile& m, uint3
     }
   } else {
     const uint4* src = reinterpret_cast<const uint4*>(a.q_rope + row * DR);
-    uint4 x[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) x[q] = ok ? src[q] : make_uint4(0, 0, 0, 0);
     const RopeAxes ax = rope_axes(G, a.q_first + i);
+    // 32 dims (16 pairs, 16 TMEM columns) at a time
+#pragma unroll 1
+    for (int c = 0; c < DR / 32; ++c) {
+      uint4 x[4];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+      for (int q = 0; q < 4; ++q) x[q] = ok ? src[4 * c + q] : make_uint4(0, 0, 0, 0);
       uint32_t v[16];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint32_t w[4] = {x[4 * c + q].x, x[4 * c + q].y, x[4 * c + q].z, x[4 * c + q].w};
+        const uint32_t w[4] = {x[q].x, x[q].y, x[q].z, x[q].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int p = 16 * c + 4 * q + e;            // RoPE pair: elements (2p, 2p + 1)
@@ -199,9 +214,16 @@ __device__ __forceinline__ void load_q(const MatArgs& a, const MatTile& m, uint3
   tmem_wait_st();
 }
 
+template <int DRV>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attend_mat_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKR,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ MatArgs a) {
+  using LY = MLay<DRV>;
+  constexpr int BN = LY::BN, DR = LY::DR, BOX = LY::BOX, NRB = LY::NRB, STAGE = LY::STAGE;
+  constexpr int PBUF = LY::PBUF, OFF_K = LY::OFF_K, OFF_KR = LY::OFF_KR, OFF_V = LY::OFF_V;
+  constexpr int OFF_P = LY::OFF_P, OFF_M = LY::OFF_M, OFF_FREQ = LY::OFF_FREQ;
+  constexpr int OFF_BAR = LY::OFF_BAR, OFF_MISC = LY::OFF_MISC;
+  constexpr uint32_t O_COL = LY::O_COL, Q_COL = LY::Q_COL, S_COL = LY::S_COL;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -242,7 +264,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  TileWalk tw;
+  TileWalk<BN> tw;
   tw.begin(a);
 
   if (warp == 8) {
@@ -268,14 +290,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_3d(sm + OFF_K + (q * NST + s) * BOX, &tmK, &bar[B_KVF + s], q * 64, m.h, r);
             tma_load_3d(sm + OFF_V + (q * NST + s) * BOX, &tmV, &bar[B_KVF + s], q * 64, m.h, r);
           }
-          tma_load_3d(sm + OFF_KR + s * BOX, &tmKR, &bar[B_KVF + s], G.Dc, (int32_t)slot0, m.b);
+#pragma unroll
+          for (int q = 0; q < NRB; ++q)
+            tma_load_3d(sm + OFF_KR + (q * NST + s) * BOX, &tmKR, &bar[B_KVF + s], G.Dc + 64 * q,
+                        (int32_t)slot0, m.b);
         }
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ score MMA issuer
-    // The scores of a block are one N=64 series into the S buffer of the warpgroup that
-    // takes it: 8 K-steps over K_h and 4 over k_R, the query as the TMEM A operand.
+    // The scores of a block are one N=BN series into the S buffer of the warpgroup that
+    // takes it: 8 K-steps over K_h and DR / 16 over k_R, the query as the TMEM A operand.
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, BN, false, false);
       bool ok = true;
@@ -299,10 +324,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mma_ts(d, tmem + Q_COL + kk * 8,
                    kd + (uint64_t)(((kk >> 2) * NST * BOX + (kk & 3) * 32) >> 4), id_qk,
                    kk > 0 ? 1u : 0u);
-          const uint64_t rd = desc_sw128(smem_u32(sm + OFF_KR + s * BOX), 16, 1024);
 #pragma unroll
-          for (int kr = 0; kr < DR / 16; ++kr)
-            mma_ts(d, tmem + Q_COL + DN / 2 + kr * 8, rd + (uint64_t)((kr * 32) >> 4), id_qk, 1u);
+          for (int kr = 0; kr < DR / 16; ++kr) {
+            const uint64_t rd =
+                desc_sw128(smem_u32(sm + OFF_KR + ((kr >> 2) * NST + s) * BOX), 16, 1024);
+            mma_ts(d, tmem + Q_COL + DN / 2 + kr * 8, rd + (uint64_t)(((kr & 3) * 32) >> 4),
+                   id_qk, 1u);
+          }
           mma_commit(&bar[B_SF + w]);
         }
         mma_commit(&bar[B_QKDONE]);
@@ -328,10 +356,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint32_t v0 = smem_u32(sm + OFF_V + s * BOX);
           const uint32_t pa = smem_u32(sm + OFF_P + pb * PBUF);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ss(tmem + O_COL, desc_sw128(pa + ks * 32, 16, 1024),
-                   desc_sw128(v0 + ks * 2048, NST * BOX, 1024), id_pv,
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            // P is K-major: rows of BN keys, 128-byte swizzle (64 keys) or 64-byte (32 keys)
+            const uint64_t pd = BN == 64 ? desc_sw128(pa + ks * 32, 16, 1024)
+                                         : desc_sw64(pa, 512) + (uint64_t)((ks * 32) >> 4);
+            mma_ss(tmem + O_COL, pd, desc_sw128(v0 + ks * 2048, NST * BOX, 1024), id_pv,
                    (jl > 0 || ks > 0) ? 1u : 0u);
+          }
           mma_commit(&bar[B_PE + pb]);
           mma_commit(&bar[B_KVE + s]);
         }
@@ -349,7 +380,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
 
     if (tw.valid(a)) {
-      load_q(a, tw.m, tmem + lane_base + Q_COL, t, wg, inv_freq);
+      load_q<DR>(a, tw.m, tmem + lane_base + Q_COL, t, wg, inv_freq);
       tc_fence_before();
       mbar_arrive(&bar[B_QREADY]);
     }
@@ -371,15 +402,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         float s[BN];
         {
-          uint32_t v[2][32];
-          tmem_ld32(tmem + lane_base + S_COL + wg * BN, v[0]);
-          tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32, v[1]);
+          uint32_t v[BN / 32][32];
+#pragma unroll
+          for (int h = 0; h < BN / 32; ++h) tmem_ld32(tmem + lane_base + S_COL + wg * BN + 32 * h, v[h]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            s[c] = __uint_as_float(v[0][c]);
-            s[32 + c] = __uint_as_float(v[1][c]);
-          }
+          for (int h = 0; h < BN / 32; ++h)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) s[32 * h + c] = __uint_as_float(v[h][c]);
         }
         tc_fence_before();
         mbar_arrive(&bar[B_SE + wg]);
@@ -461,11 +491,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        // P row t, 16-byte chunks in the 128-byte hardware swizzle (chunk ^ (row & 7))
+        // P row t, 16-byte chunks in the hardware swizzle: chunk ^ (row & 7) for 128-byte
+        // rows (64 keys), chunk ^ ((row / 2) & 3) for 64-byte rows (32 keys)
 #pragma unroll
-        for (int c = 0; c < BN / 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) * 16)) =
+        for (int c = 0; c < BN / 8; ++c) {
+          const int cs = BN == 64 ? (c ^ (t & 7)) : (c ^ ((t >> 1) & 3));
+          *reinterpret_cast<uint4*>(prow + cs * 16) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar[B_PF + wg]);
@@ -475,12 +508,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // the next tile's query may enter TMEM once this tile's score MMAs are done
       const uint32_t kph = tw.k & 1;
       {
-        TileWalk nx = tw;
+        TileWalk<BN> nx = tw;
         nx.next(a);
         if (nx.valid(a)) {
           if (!__all_sync(FULL, mbar_wait(&bar[B_QKDONE], kph, abort, a.err, 0x701, t))) break;
           tc_fence_after();
-          load_q(a, nx.m, tmem + lane_base + Q_COL, t, wg, inv_freq);
+          load_q<DR>(a, nx.m, tmem + lane_base + Q_COL, t, wg, inv_freq);
           tc_fence_before();
           mbar_arrive(&bar[B_QREADY]);
         }
@@ -537,6 +570,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+template <int DRV>
 int sm_count() {
   static std::mutex mu;
   static int cached[64] = {0};
@@ -547,8 +581,8 @@ int sm_count() {
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
     return 0;
-  if (cudaFuncSetAttribute(attend_mat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SMEM) != cudaSuccess)
+  if (cudaFuncSetAttribute(attend_mat_kernel<DRV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           MLay<DRV>::SMEM) != cudaSuccess)
     return 0;
   if (dev < 64) cached[dev] = n;
   return n;
@@ -557,19 +591,22 @@ int sm_count() {
 }  // namespace
 
 bool tc_attend_mat_supported(const Geo& g) {
-  return g.Dn == DN && g.Dr == DR && g.Dc % 128 == 0 && (int64_t)g.B * g.S < INT32_MAX;
+  return g.Dn == DN && (g.Dr == 64 || g.Dr == 512) && g.Dc % 128 == 0 &&
+         (int64_t)g.B * g.S < INT32_MAX;
 }
 
 cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, int64_t n_q,
                           int64_t q_first, const void* cache, const void* k_mat,
                           const void* v_mat, int64_t k_first, int64_t n_keys, float scale,
                           void* out, float* lse, unsigned int* err, cudaStream_t st) {
+  const bool wide = g.Dr == 512;
+  const int bn = wide ? MLay<512>::BN : MLay<64>::BN;
   CUtensorMap K, KR, V;
   {
     // K_h / V_h as (d_nope, heads, slots of all sequences): 64-dim boxes of 64 slots
     uint64_t d[3] = {(uint64_t)DN, (uint64_t)g.H, (uint64_t)g.B * g.S};
     uint64_t s[2] = {(uint64_t)DN * 2, (uint64_t)g.H * DN * 2};
-    uint32_t b[3] = {64, 1, (uint32_t)BN};
+    uint32_t b[3] = {64, 1, (uint32_t)bn};
     if (!make_tmap_bf16(&K, k_mat, 3, d, s, b)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&V, v_mat, 3, d, s, b)) return cudaErrorInvalidValue;
   }
@@ -577,10 +614,10 @@ cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, 
     // the cached rows, for their k_R columns: (row, slots, sequences)
     uint64_t d[3] = {(uint64_t)g.row, (uint64_t)g.S, (uint64_t)g.B};
     uint64_t s[2] = {(uint64_t)g.row * 2, (uint64_t)g.S * g.row * 2};
-    uint32_t b[3] = {64, (uint32_t)BN, 1};
+    uint32_t b[3] = {64, (uint32_t)bn, 1};
     if (!make_tmap_bf16(&KR, cache, 3, d, s, b)) return cudaErrorInvalidValue;
   }
-  const int nsm = sm_count();
+  const int nsm = wide ? sm_count<512>() : sm_count<64>();
   if (nsm == 0) return cudaErrorInvalidDevice;
   MatArgs a{};
   a.g = g;
@@ -597,7 +634,10 @@ cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, 
   a.err = err;
   if (a.tiles == 0) return cudaSuccess;
   const int grid = a.tiles < nsm ? a.tiles : nsm;
-  attend_mat_kernel<<<grid, NTHREADS, SMEM, st>>>(K, KR, V, a);
+  if (wide)
+    attend_mat_kernel<512><<<grid, NTHREADS, MLay<512>::SMEM, st>>>(K, KR, V, a);
+  else
+    attend_mat_kernel<64><<<grid, NTHREADS, MLay<64>::SMEM, st>>>(K, KR, V, a);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;

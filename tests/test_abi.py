@@ -149,10 +149,13 @@ def test_materialised_validation(L):
     s = _shape()
     # per-head keys and values of every ring slot, bf16
     assert L.mla_attend_materialised_workspace_size(ctypes.byref(s)) == 2 * 6240 * 32 * 128 * 2
+    # the wide positional key (d_R = 512) is supported; other RoPE widths are not
     wide = native.make_shape(C.WIDE_KEY)
-    assert L.mla_attend_materialised_workspace_size(ctypes.byref(wide)) == 0
-    assert _mat(L, wide, n_q=1560, q_first=9 * 1560, n_keys=15600, ws_bytes=1 << 30) == \
-        native.MLA_ERR_UNSUPPORTED
+    assert L.mla_attend_materialised_workspace_size(ctypes.byref(wide)) == \
+        2 * 4 * 15600 * 32 * 128 * 2
+    other = _shape(d_rope=128, rope_pairs=[16, 24, 24])
+    assert L.mla_attend_materialised_workspace_size(ctypes.byref(other)) == 0
+    assert _mat(L, other, ws_bytes=1 << 30) == native.MLA_ERR_UNSUPPORTED
     assert _mat(L, _shape(dtype=native.MLA_F32), ws_bytes=1 << 30) == native.MLA_ERR_UNSUPPORTED
     assert _mat(L, s, ws=None) == native.MLA_ERR_ARG
     assert _mat(L, s, ws_bytes=1024) == native.MLA_ERR_ARG

@@ -24,7 +24,15 @@ SMALL = [C.small_variant(C.VIDEO_CHUNK), C.small_variant(C.LONG_WINDOW),
                                                window_frames=5, chunk_frames=2,
                                                first_chunk_frame=9, ring_slots=7 * 66),
          # 66 ring slots never written (NaN): the last key block's box reaches into them
-         C.small_variant(C.VIDEO_CHUNK).scaled(name="mat_spare_slots", ring_slots=5 * 66)]
+         C.small_variant(C.VIDEO_CHUNK).scaled(name="mat_spare_slots", ring_slots=5 * 66),
+         # the wide positional key (d_R = 512: 32-key blocks): two sequences, a ragged
+         # 45-query tile; and three chunk frames (135 queries: two query blocks) over a
+         # ring the history wraps
+         C.small_variant(C.WIDE_KEY),
+         C.small_variant(C.WIDE_KEY).scaled(name="mat_wide_wrapped", chunk_frames=3,
+                                            window_frames=4, first_chunk_frame=9,
+                                            ring_slots=8 * 45)]
+WIDE_SMALL = SMALL[4]
 
 
 def run_materialised(r, with_lse=True):
@@ -55,9 +63,9 @@ def test_small_against_materialised_definition(wl, cuda_ok):
     assert np.abs(lse.cpu().numpy() - lse_ref).max() < 2e-2
 
 
-def test_small_matches_absorbed_path(cuda_ok):
+@pytest.mark.parametrize("wl", [SMALL[2], WIDE_SMALL], ids=lambda w: w.name)
+def test_small_matches_absorbed_path(wl, cuda_ok):
     """Both forms of the same attention on the GPU agree to bf16 rounding."""
-    wl = SMALL[2]
     r = P.run_chunk(P.populate(wl, seed=0))
     out, lse = run_materialised(r)
     P.tol_check(P.download(out), P.download(r.out), wl.dtype, "materialised vs absorbed")
@@ -72,7 +80,7 @@ def test_without_lse(cuda_ok):
     assert torch.equal(out_a, out_b)
 
 
-@pytest.mark.parametrize("wl", [C.VIDEO_CHUNK, C.LONG_WINDOW], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [C.VIDEO_CHUNK, C.LONG_WINDOW, C.WIDE_KEY], ids=lambda w: w.name)
 def test_full_sampled_rows(wl, cuda_ok):
     r = P.populate(wl, seed=0)
     out, lse = run_materialised(r)

@@ -777,7 +777,8 @@ def run_ours(args):
     att_ms = kernels_ms["attend"]
     achieved = fl["attend"] / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    legs = set(LEGS) if args.legs == "all" else set(args.legs.split(","))
+    legs = set(LEGS) if args.legs == "all" else \
+        set() if args.legs == "none" else set(args.legs.split(","))
     unknown = legs - set(LEGS)
     if unknown:
         raise SystemExit(f"unknown legs: {sorted(unknown)}")
@@ -910,7 +911,8 @@ def main():
                     help="the step's workload (default: the video chunk)")
     ap.add_argument("--legs", default="all",
                     help="comma-separated extra legs to run after the step (default all: "
-                         + ",".join(LEGS) + "); fewer legs make a shorter run to profile")
+                         + ",".join(LEGS) + "; or none); fewer legs make a shorter run to "
+                         "profile")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

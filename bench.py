@@ -115,6 +115,8 @@ def step_config(wl, world: int) -> dict:
             "d_model": wl.d_model, "step": "cache_write+absorb_q+attend+up_v",
             "flops_per_step": sum(step_flops(wl).values()),
             "l2": "flushed (256 MB write) before each step",
+            "per_call_times": "from as many steps again, interleaved with the timed ones, that "
+                              "record an event between the calls",
             "parallelism": f"replicas x{world} (independent sequences)"}
 
 
@@ -341,6 +343,30 @@ def time_steps(torch, fn, steps, flush, n_marks=0):
     return st, parts
 
 
+def time_steps_and_calls(torch, step, steps, flush):
+    """`steps` timed steps for the step's rate, interleaved with as many steps that record
+    an event between each of the step's calls for the per-call breakdown.  An event
+    between two kernels keeps the second from starting while the first finishes, so the
+    timed steps carry none; interleaving puts both under the same clocks.  Returns
+    (step ms list, per-call ms lists)."""
+    st, parts = [], [[] for _ in Step.STAGES]
+    for i in range(2 * steps):
+        marked = i % 2 == 1
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if marked else None
+        e0.record()
+        step.run(ev=marks)
+        e1.record()
+        torch.cuda.synchronize()
+        if marked:
+            for k in range(4):
+                parts[k].append(marks[k].elapsed_time(marks[k + 1]))
+        else:
+            st.append(e0.elapsed_time(e1))
+    return st, parts
+
+
 def materialised_leg(torch, mla, step, steps, warmup, flush, absorbed_ms):
     """The non-absorbed form of the same chunk: mla_attend_materialised (the per-head keys
     and values rebuilt from the latent, then attention in head space, output up-projected)
@@ -474,7 +500,7 @@ def workload_leg(torch, mla, name, steps, warmup, flush, peaks, device):
         step.run()
     torch.cuda.synchronize()
     with ClockSampler(device) as clocks:
-        ms, parts = time_steps(torch, lambda ev: step.run(ev=ev), steps, flush, n_marks=5)
+        ms, parts = time_steps_and_calls(torch, step, steps, flush)
     torch.cuda.synchronize()
     kms = {k: statistics.mean(v) for k, v in zip(Step.STAGES, parts)}
     fl = step_flops(wl)
@@ -758,9 +784,9 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        ms, parts = time_steps(torch, lambda ev: step.run(ev=ev), args.steps, flush, n_marks=5)
+        ms, parts = time_steps_and_calls(torch, step, args.steps, flush)
     torch.cuda.synchronize()
-    launches = mla.mla_kernel_launches() - n0
+    launches = (mla.mla_kernel_launches() - n0) // 2      # the timed steps' half
     if world > 1:
         dist.barrier()
     t_max = ranks_max(sum(ms), dist if world > 1 else None, "cuda")

@@ -2,6 +2,7 @@
 // were cut between clusters left one normalised bf16 partial output and one fp32
 // log-sum-exp per CTA half for each piece in the workspace.
 #include "attend_common.cuh"
+#include "launch.h"
 #include "tc_ptx.cuh"
 
 namespace mla {
@@ -23,6 +24,8 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CombineList cl) {
   constexpr int CROWS = 8 / CSPLIT;
   __shared__ float red[CSPLIT > 1 ? 8 * 32 * 17 : 1];     // [row][warp][lane][16 sums + w]
+  tc::grid_dep_wait();                             // the attention's partials are visible
+  tc::grid_dep_launch();
   const int i = blockIdx.x / (TM / CROWS);
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rr = wid / CSPLIT, part = wid % CSPLIT;
@@ -128,12 +131,10 @@ cudaError_t launch_combine(const AttnArgs& a, const CombineList& cl, cudaStream_
   for (int k = 0; k < cl.n; ++k)
     most = cl.piece0[k + 1] - cl.piece0[k] > most ? cl.piece0[k + 1] - cl.piece0[k] : most;
   if (most >= 32)
-    combine_kernel<8><<<(unsigned)(cl.n * TM), 256, 0, st>>>(a, cl);
-  else if (most >= 8)
-    combine_kernel<4><<<(unsigned)(cl.n * (TM / 2)), 256, 0, st>>>(a, cl);
-  else
-    combine_kernel<1><<<(unsigned)(cl.n * (TM / 8)), 256, 0, st>>>(a, cl);
-  return cudaGetLastError();
+    return launch_dependent(combine_kernel<8>, (unsigned)(cl.n * TM), 256, 0, st, 1u, a, cl);
+  if (most >= 8)
+    return launch_dependent(combine_kernel<4>, (unsigned)(cl.n * (TM / 2)), 256, 0, st, 1u, a, cl);
+  return launch_dependent(combine_kernel<1>, (unsigned)(cl.n * (TM / 8)), 256, 0, st, 1u, a, cl);
 }
 
 }  // namespace attn

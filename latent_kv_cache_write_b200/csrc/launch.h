@@ -9,6 +9,36 @@
 
 namespace mla {
 
+// Launch a kernel so that it may start while the previous kernel on the stream finishes
+// (programmatic dependent launch): its CTAs set up barriers and tensor memory, then wait
+// in grid_dep_wait before their first global access.  Hides each launch's latency and
+// prologue behind the previous kernel's tail.  cluster_x > 1 sets the cluster size of a
+// kernel that has none compiled in.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block,
+                                    size_t smem, cudaStream_t st, unsigned cluster_x,
+                                    Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Host-side count of kernels launched by the library (see mla_kernel_launches).
 void count_launches(int n);
 

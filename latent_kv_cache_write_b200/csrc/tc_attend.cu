@@ -344,6 +344,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
   cluster_sync();          // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();                               // the previous kernel's outputs are visible
+  grid_dep_launch();
 
   SegWalk sw;
   sw.begin(sc, a, blockIdx.x >> 1);
@@ -1295,13 +1297,16 @@ cudaError_t tc_attend_ring(const Geo& g, const void* q_abs, int64_t n_q, int64_t
     a.ws_lse = reinterpret_cast<float*>(a.ws_o + (size_t)2 * ncl * TM * g.Dc);
   }
   for (const Plan& p : plans) {
+    cudaError_t e;
     if (variant == 2)
-      attend_kernel<2><<<(unsigned)(2 * p.G), Lay<2>::NT, Lay<2>::SMEM, st>>>(K, KR, QR, SC, SR, a, p.sc);
+      e = launch_dependent(attend_kernel<2>, (unsigned)(2 * p.G), Lay<2>::NT, Lay<2>::SMEM, st, 1u,
+                           K, KR, QR, SC, SR, a, p.sc);
     else if (variant == 1)
-      attend_kernel<1><<<(unsigned)(2 * p.G), Lay<1>::NT, Lay<1>::SMEM, st>>>(K, KR, QR, SC, SR, a, p.sc);
+      e = launch_dependent(attend_kernel<1>, (unsigned)(2 * p.G), Lay<1>::NT, Lay<1>::SMEM, st, 1u,
+                           K, KR, QR, SC, SR, a, p.sc);
     else
-      attend_kernel<0><<<(unsigned)(2 * p.G), Lay<0>::NT, Lay<0>::SMEM, st>>>(K, KR, QR, SC, SR, a, p.sc);
-    cudaError_t e = cudaGetLastError();
+      e = launch_dependent(attend_kernel<0>, (unsigned)(2 * p.G), Lay<0>::NT, Lay<0>::SMEM, st, 1u,
+                           K, KR, QR, SC, SR, a, p.sc);
     if (e != cudaSuccess) return e;
     count_launches(1);
     if (p.cl.n > 0) {

@@ -122,6 +122,8 @@ __global__ void __launch_bounds__(GTHREADS, GSTAGES == 2 ? 2 : 1)
   if constexpr (SPLITK) cluster_sync();        // the pair's barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();                               // the previous kernel's outputs are visible
+  grid_dep_launch();
 
   auto tile_coords = [&](int t, int& m0, int& n0, int& z) {
     z = t / (nm * nn);
@@ -450,25 +452,16 @@ cudaError_t launch_st(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
     const long long slots = (long long)sm_count() * (ST == 2 ? 2 : 1);
     const int grid = (int)(tiles < slots ? tiles : slots);
     if (grid == 0) return cudaSuccess;
-    tc_gemm_kernel<ST, SK><<<grid, GTHREADS, GL::SMEM, st>>>(A, B, B2, O, q);
+    cudaError_t e = launch_dependent(tc_gemm_kernel<ST, SK>, (unsigned)grid, GTHREADS, GL::SMEM, st,
+                                     1u, A, B, B2, O, q);
+    if (e != cudaSuccess) return e;
   } else {
     // clusters of two CTAs, one cluster per tile up to one per SM pair
     const long long pairs = sm_count() / 2;
     const int nclu = (int)(tiles < pairs ? tiles : pairs);
     if (nclu == 0) return cudaSuccess;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * nclu);
-    cfg.blockDim = dim3(GTHREADS);
-    cfg.dynamicSmemBytes = GL::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<ST, SK>, A, B, B2, O, q);
+    cudaError_t e = launch_dependent(tc_gemm_kernel<ST, SK>, (unsigned)(2 * nclu), GTHREADS,
+                                     GL::SMEM, st, 2u, A, B, B2, O, q);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = cudaGetLastError();

@@ -168,6 +168,18 @@ __device__ __forceinline__ void cluster_sync() {
                ::: "memory");
 }
 
+// Programmatic dependent launch.  grid_dep_wait: wait until the grid this one follows on
+// the stream has finished and its writes are visible (at once when the launch carried no
+// such dependency); every global access of a kernel launched with launch_dependent comes
+// after it.  grid_dep_launch: let the next grid on the stream start launching (its CTAs
+// run their own prologue, then wait in grid_dep_wait for this grid to finish).
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 
 // ------------------------------------------------------------------ TMA
 

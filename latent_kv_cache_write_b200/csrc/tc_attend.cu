@@ -58,16 +58,19 @@ using namespace attn;
 //   V = 0: d_R = 64: 4 K/V stages, separate exchange and P buffers; a warpgroup hands its
 //          exchange buffer back to the peer as soon as it has read it.
 //   V = 1: d_R = 512 (the wide positional key): each CTA's 256 RoPE dims as four 64-dim
-//          boxes, Q's RoPE half (64 KB) in shared memory, 2 K/V stages of 64 KB.  P is
-//          written over the exchange buffer once the scores are read, and the PV
-//          product's commit, multicast to the peer, hands the buffer back.
+//          boxes, Q's RoPE half (64 KB) in shared memory.  The latent half of a block
+//          (32 KB, held until its PV product) and its RoPE boxes (32 KB, read by the score
+//          MMAs only) have rings of their own: 3 latent stages and one RoPE slot, which
+//          is reloaded as soon as a block's scores are done.  P is written over the
+//          exchange buffer once the scores are read, and the PV product's commit,
+//          multicast to the peer, hands the buffer back.
 //   V = 2: d_R = 64 over the low-bit ring: as V = 0 with 3 K/V stages, and the stages are
 //          not loaded but written.  TMA brings each block's packed codes and scales into a
 //          3-slot staging ring, and two warps (one key row per lane; 384 threads) write the
 //          dequantised bf16 rows into the stage in the layout the TMA loads would have.
 // K/V ring, box-major: latent box q (dims 64q..64q+63 of this CTA's half, 128-byte
-// swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of stage s at
-// OFF_KVR + (q * NST + s) * RBB.
+// swizzle) of stage s at OFF_KV + (q * NST + s) * BOXB; RoPE box q of RoPE slot r at
+// OFF_KVR + (q * NSTR + r) * RBB (NSTR = NST and r = s except for V = 1).
 // A per-block barrier completes once per use of its buffer, a per-segment one once per
 // segment; a waiter counts the uses and waits on the parity of the count.
 template <int V>
@@ -75,7 +78,8 @@ struct Lay {
   static constexpr bool WIDE = V == 1;
   static constexpr bool PACKED = V == 2;
   static constexpr int NT = PACKED ? 384 : 352;              // threads
-  static constexpr int NST = WIDE ? 2 : (PACKED ? 3 : 4);
+  static constexpr int NST = WIDE ? 3 : (PACKED ? 3 : 4);     // latent stages
+  static constexpr int NSTR = WIDE ? 1 : NST;                  // RoPE slots
   static constexpr bool MERGED = WIDE;
   static constexpr int BNK = 64;                             // keys per block
   static constexpr int BOXB = BNK * 64 * 2;                  // latent box: BNK keys x 64 dims
@@ -94,7 +98,7 @@ struct Lay {
   // row, per path)
   static constexpr int NSG = PACKED ? 3 : 0;
   static constexpr int SGC = 64 * 128, SGR = 64 * 16, SGS = 2 * 384;   // 128-byte aligned boxes
-  static constexpr int OFF_SG = OFF_KVR + NST * NRB * RBB;          // content [NSG]
+  static constexpr int OFF_SG = OFF_KVR + NSTR * NRB * RBB;         // content [NSG]
   static constexpr int OFF_SGR = OFF_SG + NSG * SGC;                // RoPE codes [NSG]
   static constexpr int OFF_SGS = OFF_SGR + NSG * SGR;               // scales [NSG]
   static constexpr int OFF_QR = (OFF_SGS + NSG * SGS + 1023) / 1024 * 1024;
@@ -116,9 +120,10 @@ struct Lay {
   static constexpr int B_PF = B_XE + 2;         // P complete, O rescaled (128)          [2]
   static constexpr int B_PE = B_PF + 2;         // PV done (MMA commit)                  [2]
   static constexpr int B_M = B_PE + 2;          // running max of a block published (128) [2]
-  static constexpr int B_KRE = B_M + 2;         // RoPE boxes of a stage free (wide; MMA commit
-                                                // after the scores)                      [NST]
-  static constexpr int B_SGF = B_KRE + NST;    // staging slot loaded (TMA)           [NSG]
+  static constexpr int B_KRE = B_M + 2;         // RoPE slot free (wide; MMA commit after the
+                                                // scores)                                [NSTR]
+  static constexpr int B_KRF = B_KRE + NSTR;    // RoPE slot loaded (wide; TMA)           [NSTR]
+  static constexpr int B_SGF = B_KRF + NSTR;   // staging slot loaded (TMA)           [NSG]
   static constexpr int B_SGE = B_SGF + NSG;    // staging slot read (64)               [NSG]
   static constexpr int NBAR = B_SGE + NSG;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -287,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
                   const __grid_constant__ CUtensorMap tmSR, const __grid_constant__ AttnArgs a,
                   const __grid_constant__ Sched sc) {
   using LY = Lay<V>;
-  constexpr int NST = LY::NST;
+  constexpr int NST = LY::NST, NSTR = LY::NSTR;
   constexpr int BN = LY::BNK, BOX_BYTES = LY::BOXB, RBOX_BYTES = LY::RBB;
   constexpr int STAGE_BYTES = LY::STAGEB, QR_BYTES = LY::QRB, XP_BYTES = LY::XPB;
   constexpr int OFF_KV = LY::OFF_KV, OFF_KVR = LY::OFF_KVR, OFF_QR = LY::OFF_QR;
@@ -312,7 +317,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar[B_KVF + s], LY::PACKED ? 64 : 1);   // TMA, or the two dequantising warps
       mbar_init(&bar[B_KVE + s], 1);
-      mbar_init(&bar[B_KRE + s], 1);
+    }
+    for (int r = 0; r < NSTR; ++r) {
+      mbar_init(&bar[B_KRE + r], 1);
+      mbar_init(&bar[LY::B_KRF + r], 1);
     }
     for (int q = 0; q < LY::NSG; ++q) {
       mbar_init(&bar[LY::B_SGF + q], 1);
@@ -497,27 +505,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
           int64_t slot0, g0;
           int valid;
           sw.tg.blk.get(j, slot0, g0, valid);
-          if constexpr (LY::WIDE) {
-            // half of a wide stage is RoPE, read only by the score MMAs: it is refilled as
-            // soon as they are done, while the latent half waits for the PV product
-            ok = mbar_wait(&bar[B_KRE + s], fph, abort, a.err, 0x109, g);
-            if (!ok) break;
-            mbar_expect_tx(&bar[B_KVF + s], STAGE_BYTES);
-#pragma unroll
-            for (int q = 0; q < LY::NRB; ++q)
-              tma_load_3d(sm + OFF_KVR + (q * NST + s) * RBOX_BYTES, &tmK, &bar[B_KVF + s],
-                          G.Dc + (int)rank * LY::RHALF + q * 64, (int32_t)slot0, sw.tg.b);
-          }
           ok = mbar_wait(&bar[B_KVE + s], fph, abort, a.err, 0x101, g);
           if (!ok) break;
-          if constexpr (!LY::WIDE) mbar_expect_tx(&bar[B_KVF + s], STAGE_BYTES);
+          mbar_expect_tx(&bar[B_KVF + s], LY::WIDE ? LY::LATB : STAGE_BYTES);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             tma_load_3d(sm + OFF_KV + (q * NST + s) * BOX_BYTES, &tmK, &bar[B_KVF + s],
                         (int)rank * HALF + q * 64, (int32_t)slot0, sw.tg.b);
-          if constexpr (!LY::WIDE)
+          if constexpr (LY::WIDE) {
+            // the block's RoPE boxes, read only by its score MMAs: the slot is refilled as
+            // soon as the previous block's scores are done
+            const int r = g % NSTR;
+            ok = mbar_wait(&bar[B_KRE + r], ((g / NSTR) & 1) ^ 1, abort, a.err, 0x109, g);
+            if (!ok) break;
+            mbar_expect_tx(&bar[LY::B_KRF + r], LY::NRB * RBOX_BYTES);
+#pragma unroll
+            for (int q = 0; q < LY::NRB; ++q)
+              tma_load_3d(sm + OFF_KVR + (q * NSTR + r) * RBOX_BYTES, &tmK, &bar[LY::B_KRF + r],
+                          G.Dc + (int)rank * LY::RHALF + q * 64, (int32_t)slot0, sw.tg.b);
+          } else {
             tma_load_3d(sm + OFF_KVR + s * RBOX_BYTES, &tmKR, &bar[B_KVF + s],
                         G.Dc + (int)rank * LY::RHALF, (int32_t)slot0, sw.tg.b);
+          }
         }
       }
     }
@@ -531,8 +540,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
     if (lane == 0) {
       prefetch_tmap(&tmQR);
       const uint32_t id_qk1 = idesc_bf16(128, BN, false, false);
-      // one score series: S columns [d, d + N) for the keys of stage s onwards
-      auto qk_series = [&](uint32_t d, int s, uint32_t id) {
+      // one score series: S columns [d, d + N) for the keys of stage s (RoPE slot r); the
+      // wide variant waits for its RoPE slot between the latent and the RoPE steps
+      auto qk_series = [&](uint32_t d, int s, int r, int g, uint32_t id) -> bool {
         // descriptor of K box column 0 at stage s; the 16-dim steps only add offsets
         const uint64_t kd = desc_sw128(smem_u32(sm + OFF_KV + s * BOX_BYTES), 16, 1024);
         mma_ts(d, tmem + Q_COL, kd, id, 0u);
@@ -541,14 +551,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
           mma_ts(d, tmem + Q_COL + kk * 8,
                  kd + (uint64_t)(((kk >> 2) * NST * BOX_BYTES + (kk & 3) * 32) >> 4), id, 1u);
         if constexpr (LY::WIDE) {
-          // 256 RoPE dims: Q's from its four 128-row boxes, K's from the stage's four boxes
+          if (!mbar_wait(&bar[LY::B_KRF + r], (g / NSTR) & 1, abort, a.err, 0x10A, g))
+            return false;
+          tc_fence_after();
+          // 256 RoPE dims: Q's from its four 128-row boxes, K's from the slot's four boxes
 #pragma unroll
           for (int kr = 0; kr < LY::RHALF / 16; ++kr) {
             const int q = kr >> 2;
             const uint64_t qd = desc_sw128(smem_u32(sm + OFF_QR + q * (TM * 128)) + (kr & 3) * 32,
                                            16, 1024);
             const uint64_t rd =
-                desc_sw128(smem_u32(sm + OFF_KVR + (q * NST + s) * RBOX_BYTES) + (kr & 3) * 32,
+                desc_sw128(smem_u32(sm + OFF_KVR + (q * NSTR + r) * RBOX_BYTES) + (kr & 3) * 32,
                            16, 1024);
             mma_ss(d, qd, rd, id, 1u);
           }
@@ -558,6 +571,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
           mma_ss(d, qd, rd, id, 1u);
           mma_ss(d, qd + 2, rd + 2, id, 1u);            // second 16-dim step: +32 bytes
         }
+        return true;
       };
       bool ok = true;
       for (; ok && sw.valid(); sw.next(a)) {
@@ -587,9 +601,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<V>::NT, 1)
           if (ok) ok = mbar_wait(&bar[B_SE + w], (q & 1) ^ 1, abort, a.err, 0x106, g);
           if (!ok) break;
           tc_fence_after();
-          qk_series(tmem + S_COL + w * BN, s, id_qk1);
+          ok = qk_series(tmem + S_COL + w * BN, s, g % NSTR, g, id_qk1);
+          if (!ok) break;
           mma_commit(&bar[B_SF + w]);
-          if constexpr (LY::WIDE) mma_commit(&bar[B_KRE + s]);
+          if constexpr (LY::WIDE) mma_commit(&bar[B_KRE + g % NSTR]);
         }
         mma_commit(&bar[B_QKDONE]);
       }

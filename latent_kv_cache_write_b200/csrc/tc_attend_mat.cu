@@ -263,6 +263,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();                               // the previous kernel's outputs are visible
+  grid_dep_launch();
 
   TileWalk<BN> tw;
   tw.begin(a);
@@ -634,11 +636,11 @@ cudaError_t tc_attend_mat(const Geo& g, const void* q_nope, const void* q_rope, 
   a.err = err;
   if (a.tiles == 0) return cudaSuccess;
   const int grid = a.tiles < nsm ? a.tiles : nsm;
-  if (wide)
-    attend_mat_kernel<512><<<grid, NTHREADS, MLay<512>::SMEM, st>>>(K, KR, V, a);
-  else
-    attend_mat_kernel<64><<<grid, NTHREADS, MLay<64>::SMEM, st>>>(K, KR, V, a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e =
+      wide ? launch_dependent(attend_mat_kernel<512>, (unsigned)grid, NTHREADS, MLay<512>::SMEM,
+                              st, 1u, K, KR, V, a)
+           : launch_dependent(attend_mat_kernel<64>, (unsigned)grid, NTHREADS, MLay<64>::SMEM,
+                              st, 1u, K, KR, V, a);
   if (e == cudaSuccess) count_launches(1);
   return e;
 }

@@ -712,16 +712,16 @@ def cpu_baseline(seconds: float = 12.0, wl=WORKLOAD):
 # were taken on (the two kernels and the headers they compile in): the value is reported
 # only while those sources are unchanged.
 ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
-                  "bytes": (72_548_608 + 17_705_216) + (19_032_320 + 4_864),
+                  "bytes": (72_825_088 + 19_140_096) + (19_032_832 + 0),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
-                          "42c52f3bf0885eaa1cc6a0ce73b17f3f4ea246879a840a92fdd2b334f8948694",
+                          "0d681a51fcb11186e077c322a23153dba8243e519e89197e62a532b7115a53ae",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
-                          "8470448cc9cefd6bf7baa6b11f034bb548d5ccce3f5dfaf611570447dd93f53a",
+                          "5e8fc3df4ef69be02af18fb893f2e454375ade78f18b76088e53fda914d78820",
                       "latent_kv_cache_write_b200/csrc/attend_common.cuh":
                           "d3ebc13662019fed51c1286a818a6dfbd805793934bf6b3a535157d562f02017",
                       "latent_kv_cache_write_b200/csrc/tc_ptx.cuh":
-                          "bb1b6e7f55916adea38d8cee629fc965ab75c4e114cd735aafa2ac6a73785d5c"}}
+                          "c4c4bb68b95a3de94a535528d9ca5cbdbd8ccbcda5f068c8974e20d715cafac1"}}
 
 
 def attend_traffic(wl=WORKLOAD):

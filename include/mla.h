@@ -23,7 +23,11 @@
  *     allocates nothing and keeps no per-call state.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
  *     and the call returns without synchronising.  Results are visible to later work
- *     on the same stream.
+ *     on the same stream.  The tensor-core kernels are launched as programmatic
+ *     dependent launches: their thread blocks may become resident while the previous
+ *     kernel on the stream finishes, but they wait for it to complete (and for its
+ *     writes to be visible) before they read or write any buffer, so stream order holds
+ *     for every buffer, whatever kernel wrote or reads it.
  *   - Arguments are validated before anything is launched; on any error status no
  *     work has been enqueued.  MLA_ERR_CUDA reports a launch failure
  *     (cudaGetLastError after the launch).

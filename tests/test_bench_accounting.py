@@ -78,3 +78,56 @@ def test_both_arms_report_one_config():
     assert cfg["workload"] == wl.name and cfg["keys"] == 6240 and cfg["queries"] == 1560
     assert cfg["flops_per_step"] == sum(bench.step_flops(wl).values())
     assert cfg["parallelism"] == "replicas x2 (independent sequences)"
+
+
+class _FakeEvent:
+    """A CUDA event stand-in whose record() takes the next tick of a shared clock."""
+    clock = [0.0]
+
+    def __init__(self, enable_timing=False):
+        self.t = None
+
+    def record(self):
+        _FakeEvent.clock[0] += 1.0
+        self.t = _FakeEvent.clock[0]
+
+    def elapsed_time(self, other):
+        return other.t - self.t
+
+
+class _FakeTorch:
+    class cuda:
+        Event = _FakeEvent
+
+        @staticmethod
+        def synchronize():
+            pass
+
+
+class _FakeStep:
+    """Records which steps carried events between their calls."""
+    def __init__(self):
+        self.calls = []
+
+    def run(self, ev=None):
+        self.calls.append(ev is not None)
+        if ev is not None:
+            for e in ev:
+                e.record()
+
+
+class _FakeFlush:
+    def zero_(self):
+        pass
+
+
+def test_timed_steps_carry_no_events_between_calls():
+    """The rate comes from steps with no event between their calls (an event there would
+    keep a kernel from starting while the previous one finishes); the per-call breakdown
+    comes from as many steps interleaved with them."""
+    step = _FakeStep()
+    ms, parts = bench.time_steps_and_calls(_FakeTorch, step, 5, _FakeFlush())
+    assert step.calls == [False, True] * 5
+    assert len(ms) == 5 and all(m == 1.0 for m in ms)     # e0 then e1 around a bare step
+    assert len(parts) == len(bench.Step.STAGES) == 4
+    assert all(len(p) == 5 and all(x == 1.0 for x in p) for p in parts)

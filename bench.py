@@ -715,7 +715,7 @@ ATTEND_TRAFFIC = {"workload": "video_chunk_bf16",
                   "bytes": (72_825_088 + 19_140_096) + (19_032_832 + 0),
                   "sources": {
                       "latent_kv_cache_write_b200/csrc/tc_attend.cu":
-                          "0d681a51fcb11186e077c322a23153dba8243e519e89197e62a532b7115a53ae",
+                          "d0c241022ed547e0bf770fb1ef23c7614fb7d20773ece53013be06c69422d3f6",
                       "latent_kv_cache_write_b200/csrc/attend_combine.cu":
                           "5e8fc3df4ef69be02af18fb893f2e454375ade78f18b76088e53fda914d78820",
                       "latent_kv_cache_write_b200/csrc/attend_common.cuh":

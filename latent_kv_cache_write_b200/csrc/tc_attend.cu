@@ -22,10 +22,12 @@
 //
 // Two softmax warpgroups take alternate key blocks, so the exchange of one block
 // overlaps the exponentials of the other; they hand the running row maximum to each
-// other through shared memory.  The buffer the peer's partial scores land in takes P
-// once they are read.  O is rescaled only when a row maximum grows by more than 8 (log2
-// units).  Masking is frame-block-causal per row; a ring that wraps is walked as two
-// contiguous slot segments.
+// other through shared memory.  In the wide variant the buffer the peer's partial scores
+// land in takes P once they are read.  O is rescaled only when a row maximum grows by
+// more than 8 (log2 units).  Masking is frame-block-causal per row; a ring that wraps is
+// walked as two contiguous slot segments.  The kernel is launched dependent on the
+// previous kernel of the stream: its prologue (barriers, TMEM) runs while that kernel
+// finishes, and it waits for it before touching any buffer.
 //
 // Scheduling is persistent and split-key ("stream-K"): the launch has one cluster per
 // pair of SMs, and the key blocks of all tiles, laid end to end, are cut into one equal
